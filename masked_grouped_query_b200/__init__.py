@@ -1,0 +1,11 @@
+"""Masked grouped-query attention forward for NVIDIA B200 (sm_100a).
+
+``make_attention(cfg)`` returns ``f(q, k, v)`` over bf16 CUDA tensors; every
+step of the computation runs in the CUDA library ``libgqa_attn.so`` behind
+the C ABI declared in ``include/gqa_attn.h``.  This package only marshals
+arguments.  Importing it does not load the library; the first call does, and
+raises if the library is missing.
+"""
+from .inputs import WORKLOADS, Workload, make_inputs  # noqa: F401
+
+__all__ = ["WORKLOADS", "Workload", "make_inputs"]
