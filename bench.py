@@ -1,0 +1,454 @@
+#!/usr/bin/env python
+"""Benchmark of the masked GQA attention forward pass (one JSON line).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl {native,reference}] [--all]
+
+A step is one call of ``gqa_attn_fwd`` over one batch of the workload -- the
+whole hot path (validate/plan, the attention kernel with its fused split-KV
+combine).  Inputs are seeded synthetic bf16 N(0,1) of the workload's shape,
+resident in HBM before timing; L2 is flushed (a 256 MiB write) between timed
+steps and each step is timed with CUDA events on the launching stream.
+
+Metric: decode workloads report K/V-read GB/s -- bytes of the keys in the
+union of the visible ranges, read once per kv head -- and prefill/encoder
+workloads report TFLOP/s over unmasked (q, k) pairs at 4 * head_dim FLOP per
+pair; both are compared with the measured peaks of the box.
+
+``--impl reference`` times the fp64 CPU oracle (the slow reference arm) on a
+bounded sample of the same workload.  Under torchrun (N > 1) each rank runs
+its own replica (independent problems, no data-path collective: weak
+scaling); the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from masked_grouped_query_b200.inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+
+DEFAULT_WORKLOAD = "gqa_decode"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------ work counts
+def is_decode(w: Workload) -> bool:
+    """Decode-class workloads (few query rows per kv head) are HBM-bound."""
+    return w.group * w.q_len <= 64
+
+
+def _first_last(w: Workload, qpos: np.ndarray):
+    first = np.zeros_like(qpos)
+    last = np.full_like(qpos, w.kv_len - 1)
+    if w.window:
+        first = np.maximum(0, qpos - w.window + 1)
+    if w.causal or w.window:
+        last = np.minimum(w.kv_len - 1, qpos)
+    return first, last
+
+
+def visible_pairs_per_head(w: Workload) -> int:
+    qpos = (w.kv_len - w.q_len) + np.arange(w.q_len, dtype=np.int64)
+    first, last = _first_last(w, qpos)
+    return int(np.maximum(0, last - first + 1).sum())
+
+
+def useful_flops(w: Workload) -> float:
+    """4 * D FLOP per unmasked (q, k) pair, logical head_dim."""
+    return 4.0 * w.head_dim * visible_pairs_per_head(w) * w.batch * w.num_q_heads
+
+
+def kv_union_keys(w: Workload) -> int:
+    qpos = (w.kv_len - w.q_len) + np.arange(w.q_len, dtype=np.int64)
+    first, last = _first_last(w, qpos)
+    ok = last >= first
+    if not ok.any():
+        return 0
+    return int(last[ok].max() - first[ok].min() + 1)
+
+
+def kv_bytes(w: Workload) -> float:
+    """K and V bytes of the visible key union, read once per kv head."""
+    return 2.0 * 2 * w.head_dim * kv_union_keys(w) * w.batch * w.num_kv_heads
+
+
+def metric_of(w: Workload):
+    if is_decode(w):
+        return ("masked-GQA attn fwd KV-read GB/s (decode)", "GB/s", kv_bytes(w) / 1e9)
+    return ("masked-GQA attn fwd TFLOP/s (prefill)", "TFLOP/s", useful_flops(w) / 1e12)
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "masked_grouped_query_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if still current."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        t = json.load(f)
+    e = t.get(workload)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.gpu = gpu_index
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        mhz, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                mhz.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for n, flag in zip(names, parts[5:9]):
+                if flag.lower() == "active":
+                    reasons.add(n)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(mhz)), "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(mhz)}
+
+
+# ------------------------------------------------------------ native arm
+def time_native(w: Workload, steps: int, warmup: int, device, dist_ctx):
+    import masked_grouped_query_b200 as mgq
+    from masked_grouped_query_b200 import _lib
+
+    lib = _lib.load()
+    q, k, v = (t.to(device) for t in make_inputs(w))
+    out = torch.empty_like(q)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    sh = torch.cuda.current_stream(device).cuda_stream
+    causal, window, cap = int(w.causal), int(w.window or 0), float(w.softcap or 0.0)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), w.batch, w.q_len,
+            w.kv_len, w.num_q_heads, w.num_kv_heads, w.head_dim, causal, window, cap)
+
+    import ctypes
+    sp = ctypes.c_void_p(sh)
+
+    def call():
+        rc = lib.gqa_attn_fwd(*args, sp)
+        if rc != 0:
+            raise RuntimeError(f"gqa_attn_fwd: {_lib.error_string(rc)}")
+
+    for _ in range(warmup):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize(device)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    dist_ctx.barrier()
+    torch.cuda.synchronize(device)
+    t0 = time.perf_counter()
+    for i in range(steps):
+        flush.zero_()
+        starts[i].record(stream)
+        call()
+        ends[i].record(stream)
+    torch.cuda.synchronize(device)
+    wall = time.perf_counter() - t0
+    dist_ctx.barrier()
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = float(np.mean(per))
+    plan = mgq.describe(w.batch, w.q_len, w.kv_len, w.num_q_heads, w.num_kv_heads,
+                        w.head_dim, w.causal, w.window, w.softcap)
+    return {"ms_mean": ms, "ms_median": float(np.median(per)), "ms_p10": float(np.percentile(per, 10)),
+            "ms_p90": float(np.percentile(per, 90)), "wall_s": wall, "launches": steps,
+            "plan": plan, "status": mgq.status()}
+
+
+def time_e2e(w: Workload, steps: int, warmup: int, device):
+    """Same metric through the host-buffer C call: H2D, kernel, D2H per step."""
+    from masked_grouped_query_b200 import _lib
+    import ctypes
+
+    lib = _lib.load()
+    qh, kh, vh = (t.pin_memory() for t in make_inputs(w))
+    oh = torch.empty(qh.shape, dtype=qh.dtype, pin_memory=True)
+    dq, dk, dv = (torch.empty(t.shape, dtype=t.dtype, device=device) for t in (qh, kh, vh))
+    do = torch.empty_like(dq)
+    sp = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    args = (qh.data_ptr(), kh.data_ptr(), vh.data_ptr(), oh.data_ptr(), dq.data_ptr(),
+            dk.data_ptr(), dv.data_ptr(), do.data_ptr(), w.batch, w.q_len, w.kv_len,
+            w.num_q_heads, w.num_kv_heads, w.head_dim, int(w.causal), int(w.window or 0),
+            float(w.softcap or 0.0), sp)
+    for _ in range(warmup):
+        rc = lib.gqa_attn_fwd_host(*args)
+        if rc != 0:
+            raise RuntimeError(f"gqa_attn_fwd_host: {_lib.error_string(rc)}")
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        rc = lib.gqa_attn_fwd_host(*args)
+        if rc != 0:
+            raise RuntimeError(f"gqa_attn_fwd_host: {_lib.error_string(rc)}")
+    e.record(stream)
+    torch.cuda.synchronize(device)
+    ms = s.elapsed_time(e) / steps
+    h2d = (qh.numel() + kh.numel() + vh.numel()) * 2
+    return ms, h2d, oh.numel() * 2
+
+
+# ------------------------------------------------------------ oracle arm
+def cpu_sample(w: Workload, budget_s: float = 12.0):
+    """Time the oracle on whole kv-head groups of the workload; returns
+    (metric value, sample description, threads, seconds)."""
+    from oracle import oracle
+
+    q, k, v = make_inputs(w)
+    threads = len(os.sched_getaffinity(0))
+    units = w.batch * w.num_kv_heads
+    g = w.group
+    name, unit, work = metric_of(w)
+    per_unit_work = work / units
+    # first a single kv-head group to size the sample
+    n_units, elapsed, done = 1, 0.0, 0
+    rows_per_unit = g * w.q_len
+    while True:
+        ids = []
+        for u in range(done, min(units, done + n_units)):
+            b, kvh = divmod(u, w.num_kv_heads)
+            for h in range(kvh * g, (kvh + 1) * g):
+                base = (b * w.num_q_heads + h) * w.q_len
+                ids.extend(range(base, base + w.q_len))
+        if not ids:
+            break
+        t0 = time.perf_counter()
+        oracle.attention_rows(q, k, v, causal=w.causal, window=w.window, softcap=w.softcap,
+                              rows=np.asarray(ids, dtype=np.int64), threads=threads)
+        dt = time.perf_counter() - t0
+        got = len(ids) // rows_per_unit
+        done += got
+        elapsed += dt
+        if elapsed >= budget_s or done >= units:
+            break
+        n_units = max(1, min(units - done, int(got * max(1.0, (budget_s - elapsed) / max(dt, 1e-6)))))
+    value = per_unit_work * done / elapsed
+    desc = (f"{done} of {units} (batch, kv head) groups ({done * rows_per_unit} query rows), "
+            f"fp64 oracle, {elapsed:.1f} s")
+    return value, desc, threads, elapsed
+
+
+# ------------------------------------------------------------ distributed
+class DistCtx:
+    def __init__(self, n_gpus: int):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", self.local))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=f"cuda:{self.local}")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--all", action="store_true", help="also time every other workload")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    w = WORKLOADS[args.workload]
+    name, unit, work = metric_of(w)
+    pk, pk_src = peaks()
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return
+        vals = []
+        desc = threads = None
+        for _ in range(args.warmup):
+            pass  # the oracle has nothing to warm up beyond the first call below
+        budget = max(1.0, 60.0 / max(1, args.steps))
+        for _ in range(args.steps):
+            val, desc, threads, _ = cpu_sample(w, budget_s=budget)
+            vals.append(val)
+        value = float(np.median(vals))
+        line = {"impl": "reference", "metric": name, "value": value, "unit": unit,
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": work / value * 1e3 if value else None,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic",
+                "config": {"workload": w.name, **{k: v for k, v in w.cfg().items() if k not in ("name",)}},
+                "cpu_baseline": {"value": value, "unit": unit, "cores": threads,
+                                 "kind": "oracle", "sample": desc},
+                "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    ctx = DistCtx(args.gpus)
+    device = torch.device("cuda", ctx.local)
+    torch.cuda.set_device(device)
+    from masked_grouped_query_b200 import build as _build
+    if not os.path.exists(_build.LIBRARY):
+        raise SystemExit("libgqa_attn.so missing: run __graft_entry__.build() first")
+
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(ctx.local)).split(",")[ctx.local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else ctx.local
+    with ClockSampler(gpu_index) as clk:
+        res = time_native(w, args.steps, args.warmup, device, ctx)
+        e2e = None
+        if not args.no_e2e:
+            e2e_steps = max(3, min(args.steps, 20))
+            e2e = time_e2e(w, e2e_steps, 3, device)
+    ms = ctx.max(res["ms_mean"])
+    value = work * ctx.world / (ms * 1e-3)
+
+    extra = {}
+    if args.all and ctx.rank == 0:
+        for other in WORKLOADS.values():
+            if other.name == w.name:
+                continue
+            r = time_native(other, max(20, args.steps // 4), args.warmup, device, _NoDist())
+            n2, u2, wk2 = metric_of(other)
+            a = wk2 / (r["ms_mean"] * 1e-3)
+            pkv = pk["hbm_gbs"] if u2 == "GB/s" else pk["bf16_tflops"]
+            extra[other.name] = {"metric": n2, "value": a, "unit": u2, "ms": r["ms_mean"],
+                                 "frac_of_peak": a / pkv, "plan": r["plan"]}
+
+    if ctx.rank == 0:
+        if unit == "GB/s":
+            peak = pk["hbm_gbs"]
+            roof = {"bound": "hbm", "achieved": work / (res["ms_mean"] * 1e-3), "peak": peak,
+                    "unit": "GB/s"}
+        else:
+            peak = pk["bf16_tflops"]
+            roof = {"bound": "tensor", "achieved": work / (res["ms_mean"] * 1e-3), "peak": peak,
+                    "unit": "TFLOP/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["peak_source"] = f"{pk_src} (MEASURED_PEAKS.json)" if pk_src == "measured" else "fallback"
+        roof["traffic"] = ncu_traffic(w.name)
+        line = {"metric": name, "value": value, "unit": unit, "n_gpus": ctx.world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": w.name,
+                           **{k: v for k, v in w.cfg().items() if k not in ("name",)},
+                           "l2": "flushed between timed steps (256 MiB write)",
+                           "parallelism": f"replica x{ctx.world}"},
+                "roofline": roof,
+                "gpu_launches": res["launches"],
+                "plan": res["plan"], "device_status": res["status"],
+                "ms_median": res["ms_median"], "ms_p10": res["ms_p10"], "ms_p90": res["ms_p90"],
+                "clocks": clk.summary()}
+        if e2e is not None:
+            ms_e2e, h2d, d2h = e2e
+            line["e2e"] = {"value": work / (ms_e2e * 1e-3), "unit": unit,
+                           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                           "ms_per_step": ms_e2e}
+        if ctx.world == 1 and not args.no_cpu:
+            val, desc, threads, _ = cpu_sample(w)
+            line["cpu_baseline"] = {"value": val, "unit": unit, "cores": threads,
+                                    "kind": "oracle", "sample": desc}
+        if extra:
+            line["other_workloads"] = extra
+        print(json.dumps(line))
+    ctx.close()
+
+
+class _NoDist:
+    def barrier(self):
+        pass
+
+
+if __name__ == "__main__":
+    main()

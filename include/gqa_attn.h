@@ -1,0 +1,166 @@
+/*
+ * gqa_attn.h -- C ABI of libgqa_attn.so: masked grouped-query attention
+ * forward pass on NVIDIA B200 (sm_100a).
+ *
+ * Operation ("TPU v6e Masked GQA Kernel Optimization", sections "What You
+ * Have" and "What You Submit"): for bf16 q (batch, num_q_heads, q_len,
+ * head_dim) and k, v (batch, num_kv_heads, kv_len, head_dim) return
+ *
+ *     o = softmax(mask(softcap(q . k^T / sqrt(head_dim)))) . v
+ *
+ * as bf16 with q's shape, for GQA ratios num_q_heads / num_kv_heads >= 1
+ * (the pages' family is 1:1 to 16:1), with an optional causal mask, an
+ * optional sliding window and an optional logit softcap s * tanh(x / s).
+ * The arguments mirror the cfg dict of that page's make_attention(cfg)
+ * entry point (its "seed" and "name" fields are harness-only and not
+ * passed).
+ *
+ * Conventions (the pages are silent on them; these are the readings used by
+ * both the CUDA path and the test oracle):
+ *   - layout: every tensor is dense, row-major, contiguous, bf16, device
+ *     memory: q and o are [batch][num_q_heads][q_len][head_dim], k and v are
+ *     [batch][num_kv_heads][kv_len][head_dim].
+ *   - q head h reads kv head h / (num_q_heads / num_kv_heads) (contiguous
+ *     groups, the same as repeat-interleaving the kv heads).
+ *   - query i sits at position qpos = kv_len - q_len + i (bottom-right
+ *     alignment of both masks).
+ *   - key j is visible iff j < kv_len
+ *         && (!causal     || j <= qpos)
+ *         && (window <= 0 || (0 <= qpos - j && qpos - j < window)).
+ *     A window of W therefore sees W keys ending at qpos, and implies j <= qpos
+ *     even without `causal`.
+ *   - logits: x = (q . k) / sqrt(head_dim) with the logical head_dim; if
+ *     softcap > 0 then x = softcap * tanh(x / softcap); masking follows.
+ *   - softmax in fp32 over the visible keys (the pages' baseline uses an fp32
+ *     softmax); P is rounded to bf16 for the P.V product on the tensor cores;
+ *     o is rounded to bf16 (round to nearest even).
+ *   - a row with no visible key returns zeros (never NaN).
+ *   - results are deterministic: the same inputs on the same device give
+ *     bitwise the same output ("Deterministic: same inputs, same output",
+ *     section "Hard Constraints").
+ *
+ * Accuracy target: |o - ref| <= 2e-2 + 2e-2 * |ref| elementwise against an
+ * fp32-or-better reference ("How It Is Judged": rtol=2e-2, atol=2e-2).
+ */
+#ifndef GQA_ATTN_H
+#define GQA_ATTN_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Return codes (negative = the call did nothing). */
+#define GQA_ATTN_OK 0
+#define GQA_ATTN_ERR_NULL_POINTER (-1) /* a tensor with elements has a NULL pointer */
+#define GQA_ATTN_ERR_MISALIGNED (-2)   /* a pointer is not 16-byte aligned */
+#define GQA_ATTN_ERR_BAD_SHAPE (-3)    /* a negative size, zero heads, or int overflow */
+#define GQA_ATTN_ERR_HEAD_RATIO (-4)   /* num_q_heads % num_kv_heads != 0 */
+#define GQA_ATTN_ERR_HEAD_DIM (-5)     /* head_dim not a multiple of 8 in [8, 256] */
+#define GQA_ATTN_ERR_SOFTCAP (-6)      /* softcap negative, NaN or infinite */
+#define GQA_ATTN_ERR_DEVICE (-7)       /* current device is not compute capability 10.x */
+#define GQA_ATTN_ERR_LAUNCH (-8)       /* a CUDA launch or copy failed */
+#define GQA_ATTN_ERR_ALLOC (-9)        /* workspace allocation failed */
+#define GQA_ATTN_ERR_TOO_LARGE (-10)   /* a dimension exceeds what the kernels index */
+#define GQA_ATTN_ERR_ALIAS (-11)       /* o overlaps q, k or v */
+#define GQA_ATTN_ERR_ARG (-12)         /* another invalid argument */
+
+/* Bits of the sticky device status word (gqa_attn_status). */
+#define GQA_ATTN_STATUS_TIMEOUT_LOADER 0x1u
+#define GQA_ATTN_STATUS_TIMEOUT_COMPUTE 0x2u
+#define GQA_ATTN_STATUS_TIMEOUT_MMA 0x4u
+#define GQA_ATTN_STATUS_TIMEOUT_SOFTMAX 0x8u
+#define GQA_ATTN_STATUS_TIMEOUT_EPILOGUE 0x10u
+#define GQA_ATTN_STATUS_TIMEOUT_SELFTEST 0x20u
+
+/*
+ * gqa_attn_fwd -- o = masked GQA attention(q, k, v).
+ *
+ * q, k, v: device pointers (read only), o: device pointer (written), layouts
+ * above, 16-byte aligned; o must not overlap q, k or v.  The caller owns all
+ * four buffers and the stream; pointers may be NULL only for tensors with no
+ * elements.  Sizes: batch, q_len, kv_len >= 0; num_q_heads, num_kv_heads >= 1
+ * with num_q_heads % num_kv_heads == 0; head_dim % 8 == 0, 8 <= head_dim <=
+ * 256.  causal: 0 or non-zero.  window <= 0 means no window.  softcap == 0
+ * means no softcap; otherwise finite and > 0.  stream: a cudaStream_t (NULL =
+ * the legacy default stream) on the current device.
+ *
+ * The call validates, plans and enqueues 1 kernel (a memset when kv_len == 0,
+ * nothing when o is empty) on `stream` and returns without synchronising.
+ * Split-KV decode partials live in a library-owned workspace per (device,
+ * stream), allocated with cudaMalloc on first need and grown on demand (so
+ * the first call of a new size synchronises the device); calls on one
+ * stream are ordered, calls on different streams do not share workspace.
+ *
+ * Returns GQA_ATTN_OK or a negative GQA_ATTN_ERR_* code.  Errors raised while
+ * the kernel runs surface at the next synchronisation (CUDA convention) and,
+ * for bounded-wait timeouts, in gqa_attn_status().
+ */
+int gqa_attn_fwd(const void* q, const void* k, const void* v, void* o, int batch, int q_len,
+                 int kv_len, int num_q_heads, int num_kv_heads, int head_dim, int causal,
+                 int window, float softcap, void* stream);
+
+/*
+ * gqa_attn_fwd_host -- the same computation for inputs and output in host
+ * memory.  q_host, k_host, v_host (read) and o_host (written) are host
+ * pointers, best page-locked (cudaHostAlloc) so the copies are asynchronous.
+ * q_dev, k_dev, v_dev, o_dev are caller-owned device buffers of the same
+ * sizes (16-byte aligned).  Enqueues on `stream`: three host-to-device copies,
+ * the attention kernel, one device-to-host copy -- one cudaMemcpyAsync per
+ * tensor -- then waits for the stream.  Returns as gqa_attn_fwd.
+ */
+int gqa_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                      void* q_dev, void* k_dev, void* v_dev, void* o_dev, int batch, int q_len,
+                      int kv_len, int num_q_heads, int num_kv_heads, int head_dim, int causal,
+                      int window, float softcap, void* stream);
+
+/*
+ * gqa_attn_describe -- the plan gqa_attn_fwd would use for these sizes on
+ * the current device, without launching anything.  Any output pointer may
+ * be NULL.  *path: 0 = nothing to do, 1 = split-KV decode kernel, 2 = tcgen05
+ * prefill kernel, 3 = zero fill (kv_len == 0).  *splits: key chunks per row
+ * block (decode) or 1.  *ctas: CTAs of the launch.  *tiles: key tiles of the
+ * widest row block.  Returns GQA_ATTN_OK or the error gqa_attn_fwd would
+ * return for these sizes.
+ */
+int gqa_attn_describe(int batch, int q_len, int kv_len, int num_q_heads, int num_kv_heads,
+                      int head_dim, int causal, int window, float softcap, int* path, int* splits,
+                      int* ctas, int* tiles);
+
+/*
+ * gqa_attn_set_override -- test and tuning knobs (process-wide).
+ * key 1: force the path (value 0 = automatic, 1 = decode, 2 = prefill);
+ * key 2: force the number of key tiles per decode split (0 = automatic).
+ * A forced path that cannot run these sizes falls back to automatic.
+ * Returns GQA_ATTN_OK or GQA_ATTN_ERR_ARG for an unknown key.
+ */
+int gqa_attn_set_override(int key, int value);
+
+/* Human-readable text for a GQA_ATTN_* return code (static storage). */
+const char* gqa_attn_error_string(int status);
+
+/*
+ * gqa_attn_status -- the sticky device status word of the current device
+ * (GQA_ATTN_STATUS_* bits, 0 = nothing happened), read with a synchronous
+ * copy; call after synchronising.  Returns -1 when it cannot be read.
+ * gqa_attn_clear_status resets it to 0 and returns GQA_ATTN_OK or an error.
+ */
+int gqa_attn_status(void);
+int gqa_attn_clear_status(void);
+
+/*
+ * gqa_attn_selftest_bounded_wait -- failure-detection self test: launches
+ * one CTA that waits on an mbarrier nothing will complete, with a wait limit
+ * of `limit_us` microseconds (1..10,000,000).  The kernel gives up, sets
+ * GQA_ATTN_STATUS_TIMEOUT_SELFTEST and returns; no trap, the context stays
+ * usable.  Enqueued on `stream`; returns GQA_ATTN_OK or an error code.
+ */
+int gqa_attn_selftest_bounded_wait(int limit_us, void* stream);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int gqa_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_ATTN_H */

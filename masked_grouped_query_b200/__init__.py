@@ -4,8 +4,12 @@
 step of the computation runs in the CUDA library ``libgqa_attn.so`` behind
 the C ABI declared in ``include/gqa_attn.h``.  This package only marshals
 arguments.  Importing it does not load the library; the first call does, and
-raises if the library is missing.
+raises if the library is missing (there is no CPU fallback).
 """
+from .attention import (attention, attention_host, clear_status, describe,  # noqa: F401
+                        make_attention, selftest_bounded_wait, set_override, status)
 from .inputs import WORKLOADS, Workload, make_inputs  # noqa: F401
 
-__all__ = ["WORKLOADS", "Workload", "make_inputs"]
+__all__ = ["attention", "attention_host", "make_attention", "describe", "set_override",
+           "status", "clear_status", "selftest_bounded_wait", "WORKLOADS", "Workload",
+           "make_inputs"]

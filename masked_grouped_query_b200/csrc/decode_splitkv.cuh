@@ -1,0 +1,362 @@
+// decode_splitkv.cuh -- memory-bound split-KV attention for short query
+// blocks (decode and multi-token decode), sm_100a.
+//
+// Work unit: one kv head of one batch element (b, kvh) and a block of up to
+// 64 "rows" -- the q rows of every q head of that GQA group, packed so each
+// K/V tile feeds all of them ("north star" (3); the grouped-query decode step
+// of "TPU v6e Masked GQA Kernel Optimization", "What You Have").  The key
+// range of a row block is cut into `splits` chunks; one CTA per chunk.
+//
+// Per CTA: one loader warp streams 64-key K and V tiles with TMA
+// (cp.async.bulk.tensor, 128-byte swizzle) into a 4-stage mbarrier ring;
+// four compute warps run S = Q K^T and O += P V on the tensor cores with
+// mma.sync m16n8k16 (bf16 in, fp32 accumulate) and an online fp32 softmax
+// with the softcap and mask fused in.  Chunks end with a log-sum-exp partial
+// (o_s, lse_s); the last CTA of a row block to finish (a ticket counter, no
+// waiting) merges the partials in fixed split order -- deterministic -- and
+// writes bf16 o.  A row with no visible key comes out as zeros.
+#pragma once
+
+#include "mask.cuh"
+#include "ptx.cuh"
+
+namespace gqa {
+
+constexpr int kDecTile = 64;        // keys per pipeline stage
+constexpr int kDecRows = 64;        // rows per CTA (at most)
+constexpr int kDecComputeWarps = 4;
+constexpr int kDecThreads = 32 * (kDecComputeWarps + 1);
+
+struct DecodeParams {
+  const __nv_bfloat16* q;
+  __nv_bfloat16* o;
+  int q_len, kv_len, head_dim;
+  int rows;            // rows per (b, kvh): group * q_len
+  int row_blocks;      // ceil(rows / 64)
+  int block_rows;      // min(64, rows): row stride of the partial buffers
+  int causal, window;
+  int use_softcap;
+  float logit_scale;   // log2(e) / sqrt(D)            (no softcap)
+  float cap_in;        // 1 / (sqrt(D) * softcap)       (softcap)
+  float cap_out;       // softcap * log2(e)             (softcap)
+  int splits;          // chunks per (unit, row block)
+  int tiles_per_split;
+  float* part_o;       // [unit][rb][split][block_rows][head_dim]  (o_s, normalised)
+  float* part_lse;     // [unit][rb][split][block_rows]            (log2 domain)
+  unsigned int* tickets;  // [unit][rb], zero between calls
+};
+
+template <int KS>
+struct DecodeCfg {
+  static constexpr int kDChunks = KS / 4;                 // 64-column TMA boxes
+  static constexpr int kBoxBytes = kDecTile * 128;        // one 64-key x 64-col box
+  static constexpr int kTileBytes = kDChunks * kBoxBytes; // K (or V) tile
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kStages = KS <= 8 ? 4 : 2;
+  static constexpr int kRingBytes = kStages * kStageBytes;
+  static constexpr int kMergeBytes = kDecComputeWarps * 16 * (KS * 16 + 2) * 4;
+  static constexpr int kSmemBytes =
+      1024 + (kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes) + 2 * kStages * 8 + 64;
+};
+
+// Byte offset of (row, 8-column chunk) inside a 128B-swizzled 64-column box.
+__device__ __forceinline__ uint32_t sw128(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <int KS>
+__global__ void __launch_bounds__(kDecThreads, 1)
+    decode_splitkv_kernel(const __grid_constant__ CUtensorMap tm_k,
+                          const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+  using C = DecodeCfg<KS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+  uint8_t* ring = smem;
+  uint64_t* full = (uint64_t*)(smem + (C::kRingBytes > C::kMergeBytes ? C::kRingBytes
+                                                                       : C::kMergeBytes));
+  uint64_t* empty = full + C::kStages;
+  int* flag = (int*)(empty + C::kStages);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Flattened grid: blockIdx.x = (unit * row_blocks + rb) * splits + split.
+  const int split = (int)(blockIdx.x % (unsigned)p.splits);
+  const int rb = (int)((blockIdx.x / (unsigned)p.splits) % (unsigned)p.row_blocks);
+  const int unit = (int)(blockIdx.x / (unsigned)p.splits / (unsigned)p.row_blocks);
+  const long long r0 = (long long)rb * kDecRows;
+  const int nr = min(kDecRows, p.rows - (int)r0);
+  const MaskSpec ms{p.q_len, p.kv_len, p.causal, p.window};
+  const KeyRange kr = key_range(ms, r0, nr, kDecTile);
+  const int t_begin = split * p.tiles_per_split;
+  const int t_end = min(kr.t_count, t_begin + p.tiles_per_split);
+  const int n_tiles = max(0, t_end - t_begin);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kDecComputeWarps);
+    }
+    fence_barrier_init();
+    flag[0] = 0;
+  }
+  __syncthreads();
+
+  if (warp == kDecComputeWarps) {
+    // ------------------------------------------------------------ loader
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_map(&tm_k);
+      tma_prefetch_map(&tm_v);
+      int issued = 0;
+      for (int t = 0; t < n_tiles; ++t) {
+        const int s = t % C::kStages;
+        if (t >= C::kStages &&
+            !mbar_wait(&empty[s], ((t / C::kStages) - 1) & 1, kStatusTimeoutProducer))
+          break;
+        uint8_t* kt = ring + s * C::kStageBytes;
+        uint8_t* vt = kt + C::kTileBytes;
+        const int key0 = (kr.t_first + t_begin + t) * kDecTile;
+        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+#pragma unroll
+        for (int c = 0; c < C::kDChunks; ++c) {
+          tma_load_3d(kt + c * C::kBoxBytes, &tm_k, &full[s], c * 64, key0, unit);
+          tma_load_3d(vt + c * C::kBoxBytes, &tm_v, &full[s], c * 64, key0, unit);
+        }
+        ++issued;
+      }
+      // Never leave with copies in flight: wait for the last loads.
+      for (int t = max(0, issued - C::kStages); t < issued; ++t)
+        mbar_wait(&full[t % C::kStages], (t / C::kStages) & 1, kStatusTimeoutProducer);
+    }
+    __syncthreads();  // (A) ring free for the merge scratch
+    __syncthreads();  // (B) merge done
+    return;
+  }
+
+  // -------------------------------------------------------------- compute
+  const int wm_count = nr <= 16 ? 1 : (nr <= 32 ? 2 : 4);
+  const int wn_count = kDecComputeWarps / wm_count;
+  const int wm = warp % wm_count, wn = warp / wm_count;
+  const int kw = kDecTile / wn_count;  // keys per warp per tile: 64, 32 or 16
+  const int D = p.head_dim;
+  const int g_row_base = wm * 16 + (lane >> 2);  // CTA row of c0/c1; +8 for c2/c3
+
+  // Q fragments (A operand, row-major 16 x 16 per k-step), straight from global.
+  uint32_t qa[KS][4];
+  {
+    const __nv_bfloat16* qb = p.q + ((long long)unit * p.rows + r0) * D;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const int row = g_row_base + ((h & 1) ? 8 : 0);
+        const int d = ks * 16 + ((h & 2) ? 8 : 0) + 2 * (lane & 3);
+        uint32_t val = 0;
+        if (row < nr && d < D) val = *(const uint32_t*)(qb + (long long)row * D + d);
+        qa[ks][h] = val;
+      }
+    }
+  }
+
+  // Per-row mask bounds (rows g_row_base and g_row_base + 8).
+  int lo[2], hi[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const long long r = r0 + g_row_base + 8 * h;
+    const int qpos = p.kv_len - p.q_len + (int)(r % p.q_len);
+    lo[h] = first_key(ms, qpos);
+    hi[h] = last_key(ms, qpos);
+  }
+
+  float o_acc[2 * KS][4];
+#pragma unroll
+  for (int n = 0; n < 2 * KS; ++n) o_acc[n][0] = o_acc[n][1] = o_acc[n][2] = o_acc[n][3] = 0.f;
+  float m_run[2] = {-INFINITY, -INFINITY};
+  float l_run[2] = {0.f, 0.f};
+  bool ok = true;
+
+  for (int t = 0; t < n_tiles && ok; ++t) {
+    const int s = t % C::kStages;
+    if (!mbar_wait(&full[s], (t / C::kStages) & 1, kStatusTimeoutConsumer)) {
+      ok = false;
+      break;
+    }
+    const uint32_t kbase = smem_u32(ring + s * C::kStageBytes);
+    const uint32_t vbase = kbase + C::kTileBytes;
+    const int key0 = (kr.t_first + t_begin + t) * kDecTile;
+    const int wkey0 = wn * kw;  // first key of this warp inside the tile
+    const bool need_mask = !(key0 >= kr.all_lo && key0 + kDecTile - 1 <= kr.all_hi);
+
+    for (int kk = 0; kk < kw / 16; ++kk) {
+      // ---- S = Q K^T for 16 keys (two n8 tiles)
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      {
+        const int mi = lane >> 3, rr = lane & 7;
+        const int key = wkey0 + kk * 16 + (mi >> 1) * 8 + rr;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const int chunk = (ks * 2 + (mi & 1)) & 7;
+          const int box = (ks * 16) / 64;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(kbase + box * C::kBoxBytes + sw128(key, chunk), b0, b1, b2, b3);
+          mma_16816(sc[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
+          mma_16816(sc[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
+        }
+      }
+      // ---- logits (log2 domain), softcap, mask
+      float x[2][4];
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float v = sc[n][e];
+          v = p.use_softcap ? p.cap_out * tanh_accurate(v * p.cap_in) : v * p.logit_scale;
+          if (need_mask) {
+            const int j = key0 + wkey0 + kk * 16 + n * 8 + 2 * (lane & 3) + (e & 1);
+            const int h = e >> 1;
+            if (j < lo[h] || j > hi[h]) v = -INFINITY;
+          }
+          x[n][e] = v;
+        }
+      // ---- online softmax update (two rows per thread, quad-wide max)
+      float mt[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float m = fmaxf(fmaxf(x[0][2 * h], x[0][2 * h + 1]), fmaxf(x[1][2 * h], x[1][2 * h + 1]));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        mt[h] = m;
+      }
+      float base[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const float m_new = fmaxf(m_run[h], mt[h]);
+        base[h] = (m_new == -INFINITY) ? 0.f : m_new;
+        const float alpha = ex2(m_run[h] - base[h]);
+        m_run[h] = m_new;
+        l_run[h] *= alpha;
+#pragma unroll
+        for (int n = 0; n < 2 * KS; ++n) {
+          o_acc[n][2 * h] *= alpha;
+          o_acc[n][2 * h + 1] *= alpha;
+        }
+      }
+      float pr[2][4];
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          pr[n][e] = ex2(x[n][e] - base[e >> 1]);
+          l_run[e >> 1] += pr[n][e];
+        }
+      const uint32_t a0 = pack_bf16(pr[0][0], pr[0][1]);
+      const uint32_t a1 = pack_bf16(pr[0][2], pr[0][3]);
+      const uint32_t a2 = pack_bf16(pr[1][0], pr[1][1]);
+      const uint32_t a3 = pack_bf16(pr[1][2], pr[1][3]);
+      // ---- O += P V for these 16 keys
+      {
+        const int mi = lane >> 3, rr = lane & 7;
+        const int key = wkey0 + kk * 16 + (mi & 1) * 8 + rr;
+#pragma unroll
+        for (int dn = 0; dn < KS; ++dn) {
+          const int chunk = (dn * 2 + (mi >> 1)) & 7;
+          const int box = (dn * 16) / 64;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(vbase + box * C::kBoxBytes + sw128(key, chunk), b0, b1, b2, b3);
+          mma_16816(o_acc[2 * dn], a0, a1, a2, a3, b0, b1);
+          mma_16816(o_acc[2 * dn + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+
+  // l is per-thread partial over its columns: reduce across the quad.
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 1);
+    l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 2);
+  }
+
+  // ---- merge the key-slices of the warps through shared memory
+  __syncthreads();  // (A) ring drained and no longer read: reuse it as merge scratch
+  const int DP = KS * 16;  // padded head dim
+  float* mrg = (float*)smem;
+  {
+    const int slot = wn * wm_count + wm;  // 0..3
+    float* so = mrg + slot * 16 * (DP + 2);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = (lane >> 2) + 8 * h;
+      float* row = so + r * (DP + 2);
+#pragma unroll
+      for (int n = 0; n < 2 * KS; ++n) {
+        row[n * 8 + 2 * (lane & 3)] = o_acc[n][2 * h];
+        row[n * 8 + 2 * (lane & 3) + 1] = o_acc[n][2 * h + 1];
+      }
+      if ((lane & 3) == 0) {
+        row[DP] = m_run[h];
+        row[DP + 1] = l_run[h];
+      }
+    }
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(kDecComputeWarps * 32) : "memory");
+
+  const bool direct = p.splits == 1;
+  const long long prow0 = (((long long)unit * p.row_blocks + rb) * p.splits + split) * p.block_rows;
+  for (int idx = threadIdx.x; idx < nr * D; idx += kDecComputeWarps * 32) {
+    const int row = idx / D, d = idx - (idx / D) * D;
+    const int rwm = row >> 4, r = row & 15;
+    float M = -INFINITY;
+    for (int w = 0; w < wn_count; ++w)
+      M = fmaxf(M, mrg[((w * wm_count + rwm) * 16 + r) * (DP + 2) + DP]);
+    const float Mb = (M == -INFINITY) ? 0.f : M;
+    float L = 0.f, O = 0.f;
+    for (int w = 0; w < wn_count; ++w) {
+      const float* row_p = mrg + ((w * wm_count + rwm) * 16 + r) * (DP + 2);
+      const float f = ex2(row_p[DP] - Mb);
+      L += f * row_p[DP + 1];
+      O += f * row_p[d];
+    }
+    const float o_val = L > 0.f ? O / L : 0.f;
+    if (direct) {
+      p.o[((long long)unit * p.rows + r0 + row) * D + d] = __float2bfloat16_rn(o_val);
+    } else {
+      p.part_o[(prow0 + row) * D + d] = o_val;
+      if (d == 0) p.part_lse[prow0 + row] = L > 0.f ? M + log2f(L) : -INFINITY;
+    }
+  }
+  __syncthreads();  // (B) pairs with the loader's second barrier
+  if (direct) return;
+
+  // ---- last CTA of this row block merges the split partials
+  __threadfence();
+  asm volatile("bar.sync 1, %0;" ::"r"(kDecComputeWarps * 32) : "memory");
+  if (threadIdx.x == 0) {
+    const unsigned int ticket = atomicAdd(&p.tickets[unit * p.row_blocks + rb], 1u);
+    flag[0] = (ticket == (unsigned)p.splits - 1) ? 1 : 0;
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(kDecComputeWarps * 32) : "memory");
+  if (!flag[0]) return;
+  __threadfence();
+  const long long pbase = ((long long)unit * p.row_blocks + rb) * p.splits * p.block_rows;
+  for (int idx = threadIdx.x; idx < nr * D; idx += kDecComputeWarps * 32) {
+    const int row = idx / D, d = idx - (idx / D) * D;
+    float M = -INFINITY;
+    for (int s = 0; s < p.splits; ++s)
+      M = fmaxf(M, __ldcg(&p.part_lse[pbase + (long long)s * p.block_rows + row]));
+    float L = 0.f, O = 0.f;
+    if (M != -INFINITY) {
+      for (int s = 0; s < p.splits; ++s) {
+        const long long pr = pbase + (long long)s * p.block_rows + row;
+        const float f = ex2(__ldcg(&p.part_lse[pr]) - M);
+        L += f;
+        O += f * __ldcg(&p.part_o[pr * D + d]);
+      }
+    }
+    const float o_val = L > 0.f ? O / L : 0.f;
+    p.o[((long long)unit * p.rows + r0 + row) * D + d] = __float2bfloat16_rn(o_val);
+  }
+  if (threadIdx.x == 0) p.tickets[unit * p.row_blocks + rb] = 0u;  // ready for the next call
+}
+
+}  // namespace gqa

@@ -1,0 +1,450 @@
+// gqa_attn.cu -- host side of libgqa_attn.so: argument validation, planning,
+// tensor maps, workspace and launches behind the C ABI of gqa_attn.h.
+//
+// Single translation unit: the kernels are included below.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "gqa_attn.h"
+#include "status.cuh"
+#include "ptx.cuh"
+#include "mask.cuh"
+#include "decode_splitkv.cuh"
+#include "selftest.cuh"
+
+namespace {
+
+using namespace gqa;
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------------ device
+struct DeviceInfo {
+  bool probed = false;
+  int sms = 0, major = 0, minor = 0;
+  int smem_optin = 0;
+  bool decode_attr[4] = {false, false, false, false};
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[64];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::atomic<int> g_force_path{0};
+std::atomic<int> g_force_tps{0};
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GQA_ATTN_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.probed) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess)
+      return GQA_ATTN_ERR_DEVICE;
+    d.probed = true;
+  }
+  if (d.major != 10) return GQA_ATTN_ERR_DEVICE;
+  if (!g_encode) {
+    cudaDriverEntryPointQueryResult q;
+    void* fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || fn == nullptr)
+      return GQA_ATTN_ERR_DEVICE;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  }
+  *out = &d;
+  return GQA_ATTN_OK;
+}
+
+// ------------------------------------------------------------------ problem
+struct Problem {
+  int batch, q_len, kv_len, hq, hkv, d, causal, window;
+  float softcap;
+  int group;
+  long long units;  // batch * hkv
+  long long rows;   // group * q_len  (rows per unit)
+};
+
+int validate(int batch, int q_len, int kv_len, int hq, int hkv, int d, int causal, int window,
+             float softcap, Problem* pr) {
+  if (batch < 0 || q_len < 0 || kv_len < 0 || hq < 1 || hkv < 1) return GQA_ATTN_ERR_BAD_SHAPE;
+  if (hq % hkv != 0) return GQA_ATTN_ERR_HEAD_RATIO;
+  if (d < 8 || d > 256 || d % 8 != 0) return GQA_ATTN_ERR_HEAD_DIM;
+  if (!(softcap >= 0.0f) || std::isinf(softcap)) return GQA_ATTN_ERR_SOFTCAP;
+  pr->batch = batch;
+  pr->q_len = q_len;
+  pr->kv_len = kv_len;
+  pr->hq = hq;
+  pr->hkv = hkv;
+  pr->d = d;
+  pr->causal = causal ? 1 : 0;
+  pr->window = window > 0 ? window : 0;
+  pr->softcap = softcap;
+  pr->group = hq / hkv;
+  pr->units = (long long)batch * hkv;
+  pr->rows = (long long)pr->group * q_len;
+  // Index limits: element offsets are 64-bit, rows per unit and TMA
+  // coordinates are 32-bit, the flattened grid is < 2^31.
+  const long long q_elems = (long long)batch * hq * (long long)q_len * d;
+  const long long kv_elems = (long long)batch * hkv * (long long)kv_len * d;
+  if (pr->rows > 0x7fffffffLL || pr->units > 0x7fffffffLL || q_elems < 0 || kv_elems < 0 ||
+      (long long)batch * hq > (1LL << 40) || q_elems > (1LL << 56) || kv_elems > (1LL << 56))
+    return GQA_ATTN_ERR_TOO_LARGE;
+  return GQA_ATTN_OK;
+}
+
+// ------------------------------------------------------------------ plan
+enum Path { kPathNone = 0, kPathDecode = 1, kPathPrefill = 2, kPathZero = 3 };
+
+struct Plan {
+  int path = kPathNone;
+  int splits = 1, tps = 1;
+  int row_blocks = 0, block_rows = 0;
+  int ks = 8;
+  int max_tiles = 0;
+  long long ctas = 0;
+  size_t ws_bytes = 0;
+  size_t off_lse = 0, off_tickets = 0;
+};
+
+inline long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+int plan_decode(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
+  pl->path = kPathDecode;
+  pl->ks = pr.d <= 64 ? 4 : pr.d <= 128 ? 8 : pr.d <= 192 ? 12 : 16;
+  pl->row_blocks = (int)ceil_div(pr.rows, kDecRows);
+  pl->block_rows = (int)(pr.rows < kDecRows ? pr.rows : kDecRows);
+  const MaskSpec ms{pr.q_len, pr.kv_len, pr.causal, pr.window};
+  int max_tiles = 0;
+  for (int rb = 0; rb < pl->row_blocks; ++rb) {
+    const long long r0 = (long long)rb * kDecRows;
+    const int nr = (int)((pr.rows - r0) < kDecRows ? (pr.rows - r0) : kDecRows);
+    const KeyRange kr = key_range(ms, r0, nr, kDecTile);
+    if (kr.t_count > max_tiles) max_tiles = kr.t_count;
+  }
+  pl->max_tiles = max_tiles;
+  const long long base = pr.units * pl->row_blocks;
+  int tps;
+  const int forced = g_force_tps.load();
+  if (max_tiles == 0) {
+    tps = 1;
+  } else if (forced > 0) {
+    tps = forced;
+  } else {
+    const long long want = ceil_div(8LL * dev.sms, base);
+    tps = (int)ceil_div(max_tiles, want < 1 ? 1 : want);
+    if (tps < 4) tps = 4;
+  }
+  if (tps > max_tiles && max_tiles > 0) tps = max_tiles;
+  pl->tps = tps;
+  pl->splits = max_tiles == 0 ? 1 : (int)ceil_div(max_tiles, tps);
+  pl->ctas = base * pl->splits;
+  if (pl->ctas > 0x7fffffffLL) return GQA_ATTN_ERR_TOO_LARGE;
+  if (pl->splits > 1) {
+    const size_t prow = (size_t)base * pl->splits * pl->block_rows;
+    const size_t o_bytes = align256(prow * pr.d * sizeof(float));
+    const size_t lse_bytes = align256(prow * sizeof(float));
+    pl->off_lse = o_bytes;
+    pl->off_tickets = o_bytes + lse_bytes;
+    pl->ws_bytes = o_bytes + lse_bytes + align256((size_t)base * sizeof(unsigned int));
+  }
+  return GQA_ATTN_OK;
+}
+
+int make_plan(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
+  if (pr.batch == 0 || pr.q_len == 0) {
+    pl->path = kPathNone;
+    return GQA_ATTN_OK;
+  }
+  if (pr.kv_len == 0) {
+    pl->path = kPathZero;
+    return GQA_ATTN_OK;
+  }
+  return plan_decode(pr, dev, pl);
+}
+
+// ------------------------------------------------------------------ workspace
+struct Workspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+// Workspace of at least `bytes` for (current device, stream).  The ticket
+// region [off_tickets, end) must read as zero: new memory is cleared on the
+// stream; kernels leave their tickets at zero.
+int get_workspace(cudaStream_t stream, size_t bytes, void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ATTN_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  Workspace& ws = g_ws[std::make_pair(dev, stream)];
+  if (ws.bytes < bytes) {
+    if (ws.ptr) {
+      cudaStreamSynchronize(stream);
+      cudaFree(ws.ptr);
+      ws.ptr = nullptr;
+      ws.bytes = 0;
+    }
+    const size_t want = bytes + bytes / 4;
+    if (cudaMalloc(&ws.ptr, want) != cudaSuccess) {
+      cudaGetLastError();
+      return GQA_ATTN_ERR_ALLOC;
+    }
+    if (cudaMemsetAsync(ws.ptr, 0, want, stream) != cudaSuccess) return GQA_ATTN_ERR_LAUNCH;
+    ws.bytes = want;
+  }
+  *out = ws.ptr;
+  return GQA_ATTN_OK;
+}
+
+// ------------------------------------------------------------------ TMA maps
+// 3-D bf16 view [outer][rows][cols] with a (64 cols x box_rows x 1) box,
+// 128-byte swizzle; out-of-range elements read as zero.
+int encode_map(CUtensorMap* map, const void* base, int cols, long long rows, long long outer,
+               int box_rows) {
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)outer};
+  cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * 2 * (cuuint64_t)rows};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? GQA_ATTN_OK : GQA_ATTN_ERR_LAUNCH;
+}
+
+// ------------------------------------------------------------------ launches
+template <int KS>
+int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
+                     const void* k, const void* v, void* o, void* ws, cudaStream_t stream) {
+  using C = DecodeCfg<KS>;
+  const int slot = KS / 4 - 1;
+  if (!dev.decode_attr[slot]) {
+    if (cudaFuncSetAttribute(decode_splitkv_kernel<KS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
+      return GQA_ATTN_ERR_LAUNCH;
+    dev.decode_attr[slot] = true;
+  }
+  CUtensorMap tk, tv;
+  if (encode_map(&tk, k, pr.d, pr.kv_len, pr.units, kDecTile) != GQA_ATTN_OK ||
+      encode_map(&tv, v, pr.d, pr.kv_len, pr.units, kDecTile) != GQA_ATTN_OK)
+    return GQA_ATTN_ERR_LAUNCH;
+  DecodeParams p;
+  p.q = (const __nv_bfloat16*)q;
+  p.o = (__nv_bfloat16*)o;
+  p.q_len = pr.q_len;
+  p.kv_len = pr.kv_len;
+  p.head_dim = pr.d;
+  p.rows = (int)pr.rows;
+  p.row_blocks = pl.row_blocks;
+  p.block_rows = pl.block_rows;
+  p.causal = pr.causal;
+  p.window = pr.window;
+  p.use_softcap = pr.softcap > 0.f ? 1 : 0;
+  const float rs = 1.0f / std::sqrt((float)pr.d);
+  p.logit_scale = kLog2e * rs;
+  p.cap_in = p.use_softcap ? rs / pr.softcap : 0.f;
+  p.cap_out = p.use_softcap ? pr.softcap * kLog2e : 0.f;
+  p.splits = pl.splits;
+  p.tiles_per_split = pl.tps;
+  p.part_o = (float*)ws;
+  p.part_lse = ws ? (float*)((char*)ws + pl.off_lse) : nullptr;
+  p.tickets = ws ? (unsigned int*)((char*)ws + pl.off_tickets) : nullptr;
+  decode_splitkv_kernel<KS><<<dim3((unsigned)pl.ctas), kDecThreads, C::kSmemBytes, stream>>>(
+      tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? GQA_ATTN_OK : GQA_ATTN_ERR_LAUNCH;
+}
+
+int launch_decode(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
+                  const void* k, const void* v, void* o, void* ws, cudaStream_t stream) {
+  switch (pl.ks) {
+    case 4: return launch_decode_ks<4>(pr, pl, dev, q, k, v, o, ws, stream);
+    case 8: return launch_decode_ks<8>(pr, pl, dev, q, k, v, o, ws, stream);
+    case 12: return launch_decode_ks<12>(pr, pl, dev, q, k, v, o, ws, stream);
+    default: return launch_decode_ks<16>(pr, pl, dev, q, k, v, o, ws, stream);
+  }
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  if (!a || !b || na == 0 || nb == 0) return false;
+  const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+  return x < y + nb && y < x + na;
+}
+
+int check_pointers(const Problem& pr, const void* q, const void* k, const void* v,
+                   const void* o) {
+  const size_t q_bytes = (size_t)pr.batch * pr.hq * (size_t)pr.q_len * pr.d * 2;
+  const size_t kv_bytes = (size_t)pr.batch * pr.hkv * (size_t)pr.kv_len * pr.d * 2;
+  if (q_bytes && (!q || !o)) return GQA_ATTN_ERR_NULL_POINTER;
+  if (kv_bytes && (!k || !v)) return GQA_ATTN_ERR_NULL_POINTER;
+  if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o) & 15u)
+    return GQA_ATTN_ERR_MISALIGNED;
+  if (overlaps(o, q_bytes, q, q_bytes) || overlaps(o, q_bytes, k, kv_bytes) ||
+      overlaps(o, q_bytes, v, kv_bytes))
+    return GQA_ATTN_ERR_ALIAS;
+  return GQA_ATTN_OK;
+}
+
+int run(const Problem& pr, const void* q, const void* k, const void* v, void* o,
+        cudaStream_t stream) {
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc != GQA_ATTN_OK) return rc;
+  Plan pl;
+  rc = make_plan(pr, *dev, &pl);
+  if (rc != GQA_ATTN_OK) return rc;
+  switch (pl.path) {
+    case kPathNone:
+      return GQA_ATTN_OK;
+    case kPathZero: {
+      const size_t bytes = (size_t)pr.batch * pr.hq * (size_t)pr.q_len * pr.d * 2;
+      return cudaMemsetAsync(o, 0, bytes, stream) == cudaSuccess ? GQA_ATTN_OK
+                                                                 : GQA_ATTN_ERR_LAUNCH;
+    }
+    default: {
+      void* ws = nullptr;
+      if (pl.ws_bytes) {
+        rc = get_workspace(stream, pl.ws_bytes, &ws);
+        if (rc != GQA_ATTN_OK) return rc;
+      }
+      return launch_decode(pr, pl, *dev, q, k, v, o, ws, stream);
+    }
+  }
+}
+
+}  // namespace
+
+// ==================================================================== C ABI
+extern "C" {
+
+int gqa_attn_fwd(const void* q, const void* k, const void* v, void* o, int batch, int q_len,
+                 int kv_len, int num_q_heads, int num_kv_heads, int head_dim, int causal,
+                 int window, float softcap, void* stream) {
+  Problem pr;
+  int rc = validate(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, causal, window,
+                    softcap, &pr);
+  if (rc != GQA_ATTN_OK) return rc;
+  rc = check_pointers(pr, q, k, v, o);
+  if (rc != GQA_ATTN_OK) return rc;
+  return run(pr, q, k, v, o, (cudaStream_t)stream);
+}
+
+int gqa_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                      void* q_dev, void* k_dev, void* v_dev, void* o_dev, int batch, int q_len,
+                      int kv_len, int num_q_heads, int num_kv_heads, int head_dim, int causal,
+                      int window, float softcap, void* stream) {
+  Problem pr;
+  int rc = validate(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, causal, window,
+                    softcap, &pr);
+  if (rc != GQA_ATTN_OK) return rc;
+  rc = check_pointers(pr, q_dev, k_dev, v_dev, o_dev);
+  if (rc != GQA_ATTN_OK) return rc;
+  const size_t q_bytes = (size_t)pr.batch * pr.hq * (size_t)pr.q_len * pr.d * 2;
+  const size_t kv_bytes = (size_t)pr.batch * pr.hkv * (size_t)pr.kv_len * pr.d * 2;
+  if ((q_bytes && (!q_host || !o_host)) || (kv_bytes && (!k_host || !v_host)))
+    return GQA_ATTN_ERR_NULL_POINTER;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (q_bytes && cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return GQA_ATTN_ERR_LAUNCH;
+  if (kv_bytes &&
+      (cudaMemcpyAsync(k_dev, k_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+       cudaMemcpyAsync(v_dev, v_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess))
+    return GQA_ATTN_ERR_LAUNCH;
+  rc = run(pr, q_dev, k_dev, v_dev, o_dev, s);
+  if (rc != GQA_ATTN_OK) return rc;
+  if (q_bytes && cudaMemcpyAsync(o_host, o_dev, q_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return GQA_ATTN_ERR_LAUNCH;
+  return cudaStreamSynchronize(s) == cudaSuccess ? GQA_ATTN_OK : GQA_ATTN_ERR_LAUNCH;
+}
+
+int gqa_attn_describe(int batch, int q_len, int kv_len, int num_q_heads, int num_kv_heads,
+                      int head_dim, int causal, int window, float softcap, int* path, int* splits,
+                      int* ctas, int* tiles) {
+  Problem pr;
+  int rc = validate(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, causal, window,
+                    softcap, &pr);
+  if (rc != GQA_ATTN_OK) return rc;
+  DeviceInfo* dev = nullptr;
+  rc = device_info(&dev);
+  if (rc != GQA_ATTN_OK) return rc;
+  Plan pl;
+  rc = make_plan(pr, *dev, &pl);
+  if (rc != GQA_ATTN_OK) return rc;
+  if (path) *path = pl.path;
+  if (splits) *splits = pl.splits;
+  if (ctas) *ctas = (int)pl.ctas;
+  if (tiles) *tiles = pl.max_tiles;
+  return GQA_ATTN_OK;
+}
+
+int gqa_attn_set_override(int key, int value) {
+  if (key == 1) {
+    g_force_path.store(value);
+    return GQA_ATTN_OK;
+  }
+  if (key == 2) {
+    g_force_tps.store(value > 0 ? value : 0);
+    return GQA_ATTN_OK;
+  }
+  return GQA_ATTN_ERR_ARG;
+}
+
+const char* gqa_attn_error_string(int status) {
+  switch (status) {
+    case GQA_ATTN_OK: return "ok";
+    case GQA_ATTN_ERR_NULL_POINTER: return "null pointer for a tensor with elements";
+    case GQA_ATTN_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case GQA_ATTN_ERR_BAD_SHAPE: return "invalid size (negative, or zero heads)";
+    case GQA_ATTN_ERR_HEAD_RATIO: return "num_q_heads is not a multiple of num_kv_heads";
+    case GQA_ATTN_ERR_HEAD_DIM: return "head_dim must be a multiple of 8 in [8, 256]";
+    case GQA_ATTN_ERR_SOFTCAP: return "softcap must be finite and >= 0";
+    case GQA_ATTN_ERR_DEVICE: return "current device is not an sm_100 (B200-class) GPU";
+    case GQA_ATTN_ERR_LAUNCH: return "CUDA launch or copy failed";
+    case GQA_ATTN_ERR_ALLOC: return "workspace allocation failed";
+    case GQA_ATTN_ERR_TOO_LARGE: return "problem exceeds the kernels' index range";
+    case GQA_ATTN_ERR_ALIAS: return "output overlaps an input";
+    case GQA_ATTN_ERR_ARG: return "invalid argument";
+    default: return "unknown status";
+  }
+}
+
+int gqa_attn_status(void) {
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, gqa::g_gqa_status, sizeof v) != cudaSuccess) return -1;
+  return (int)v;
+}
+
+int gqa_attn_clear_status(void) {
+  const uint32_t z = 0;
+  return cudaMemcpyToSymbol(gqa::g_gqa_status, &z, sizeof z) == cudaSuccess ? GQA_ATTN_OK
+                                                                             : GQA_ATTN_ERR_LAUNCH;
+}
+
+int gqa_attn_selftest_bounded_wait(int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 10000000) return GQA_ATTN_ERR_ARG;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc != GQA_ATTN_OK) return rc;
+  gqa::selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((unsigned long long)limit_us *
+                                                                 1000ull);
+  return cudaGetLastError() == cudaSuccess ? GQA_ATTN_OK : GQA_ATTN_ERR_LAUNCH;
+}
+
+int gqa_attn_version(void) { return 100; }
+
+}  // extern "C"
