@@ -52,7 +52,7 @@ struct DecodeCfg {
   static constexpr int kBoxBytes = kDecTile * 128;        // one 64-key x 64-col box
   static constexpr int kTileBytes = kDChunks * kBoxBytes; // K (or V) tile
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = KS <= 8 ? 4 : 2;
+  static constexpr int kStages = KS <= 8 ? 3 : 2;
   static constexpr int kRingBytes = kStages * kStageBytes;
   static constexpr int kMergeBytes = kDecComputeWarps * 16 * (KS * 16 + 2) * 4;
   static constexpr int kSmemBytes =
@@ -338,23 +338,43 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   asm volatile("bar.sync 1, %0;" ::"r"(kDecComputeWarps * 32) : "memory");
   if (!flag[0]) return;
   __threadfence();
+  // Split weights w_s = 2^(lse_s - M) / sum_s 2^(lse_s - M) per row, in the
+  // (now idle) ring; then every thread streams float4 chunks of the partials
+  // with independent loads.
   const long long pbase = ((long long)unit * p.row_blocks + rb) * p.splits * p.block_rows;
-  for (int idx = threadIdx.x; idx < nr * D; idx += kDecComputeWarps * 32) {
-    const int row = idx / D, d = idx - (idx / D) * D;
+  float* wgt = (float*)smem;  // [split][nr]
+  for (int row = threadIdx.x; row < nr; row += kDecComputeWarps * 32) {
     float M = -INFINITY;
     for (int s = 0; s < p.splits; ++s)
       M = fmaxf(M, __ldcg(&p.part_lse[pbase + (long long)s * p.block_rows + row]));
-    float L = 0.f, O = 0.f;
-    if (M != -INFINITY) {
-      for (int s = 0; s < p.splits; ++s) {
-        const long long pr = pbase + (long long)s * p.block_rows + row;
-        const float f = ex2(__ldcg(&p.part_lse[pr]) - M);
-        L += f;
-        O += f * __ldcg(&p.part_o[pr * D + d]);
-      }
+    float L = 0.f;
+    for (int s = 0; s < p.splits; ++s) {
+      const float f = M == -INFINITY
+                          ? 0.f
+                          : ex2(__ldcg(&p.part_lse[pbase + (long long)s * p.block_rows + row]) - M);
+      wgt[s * nr + row] = f;
+      L += f;
     }
-    const float o_val = L > 0.f ? O / L : 0.f;
-    p.o[((long long)unit * p.rows + r0 + row) * D + d] = __float2bfloat16_rn(o_val);
+    const float inv = L > 0.f ? 1.0f / L : 0.f;
+    for (int s = 0; s < p.splits; ++s) wgt[s * nr + row] *= inv;
+  }
+  asm volatile("bar.sync 1, %0;" ::"r"(kDecComputeWarps * 32) : "memory");
+  const int d4 = D / 4;
+  for (int idx = threadIdx.x; idx < nr * d4; idx += kDecComputeWarps * 32) {
+    const int row = idx / d4, c = idx - (idx / d4) * d4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int s = 0; s < p.splits; ++s) {
+      const float w = wgt[s * nr + row];
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(
+          p.part_o + (pbase + (long long)s * p.block_rows + row) * D) + c);
+      acc.x += w * v.x;
+      acc.y += w * v.y;
+      acc.z += w * v.z;
+      acc.w += w * v.w;
+    }
+    uint2 packed = make_uint2(pack_bf16(acc.x, acc.y), pack_bf16(acc.z, acc.w));
+    *reinterpret_cast<uint2*>(p.o + ((long long)unit * p.rows + r0 + row) * D + 4 * c) = packed;
   }
   if (threadIdx.x == 0) p.tickets[unit * p.row_blocks + rb] = 0u;  // ready for the next call
 }

@@ -19,6 +19,7 @@
 #include "ptx.cuh"
 #include "mask.cuh"
 #include "decode_splitkv.cuh"
+#include "prefill_sm100.cuh"
 #include "selftest.cuh"
 
 namespace {
@@ -33,6 +34,7 @@ struct DeviceInfo {
   int sms = 0, major = 0, minor = 0;
   int smem_optin = 0;
   bool decode_attr[4] = {false, false, false, false};
+  bool prefill_attr[2] = {false, false};
 };
 
 std::mutex g_mu;
@@ -116,8 +118,11 @@ struct Plan {
   int ks = 8;
   int max_tiles = 0;
   long long ctas = 0;
-  size_t ws_bytes = 0;
-  size_t off_lse = 0, off_tickets = 0;
+  int dch = 2, d_pad = 128;           // prefill: TMA boxes per tile, padded head_dim
+  int tiles_per_unit = 0, pairs_per_unit = 0, pair_heads = 0;
+  size_t ws_bytes = 0;      // split partials (o_s, lse_s)
+  size_t off_lse = 0;
+  size_t ticket_bytes = 0;  // split tickets (kept zero between calls)
 };
 
 inline long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
@@ -150,6 +155,8 @@ int plan_decode(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
     if (tps < 4) tps = 4;
   }
   if (tps > max_tiles && max_tiles > 0) tps = max_tiles;
+  // The combine keeps splits x rows weights in shared memory: at most 256 splits.
+  if (max_tiles > 0 && ceil_div(max_tiles, tps) > 256) tps = (int)ceil_div(max_tiles, 256);
   pl->tps = tps;
   pl->splits = max_tiles == 0 ? 1 : (int)ceil_div(max_tiles, tps);
   pl->ctas = base * pl->splits;
@@ -159,9 +166,31 @@ int plan_decode(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
     const size_t o_bytes = align256(prow * pr.d * sizeof(float));
     const size_t lse_bytes = align256(prow * sizeof(float));
     pl->off_lse = o_bytes;
-    pl->off_tickets = o_bytes + lse_bytes;
-    pl->ws_bytes = o_bytes + lse_bytes + align256((size_t)base * sizeof(unsigned int));
+    pl->ws_bytes = o_bytes + lse_bytes;
+    pl->ticket_bytes = align256((size_t)base * sizeof(unsigned int));
   }
+  return GQA_ATTN_OK;
+}
+
+int plan_prefill(const Problem& pr, Plan* pl) {
+  pl->path = kPathPrefill;
+  pl->dch = pr.d <= 64 ? 1 : 2;
+  pl->d_pad = (pr.d + 15) / 16 * 16;
+  pl->tiles_per_unit = (int)ceil_div(pr.rows, kPfM);
+  pl->pair_heads = (pr.q_len % kPfM == 0 && pr.group % 2 == 0) ? 1 : 0;
+  pl->pairs_per_unit = pl->pair_heads ? (pr.group / 2) * (pr.q_len / kPfM)
+                                      : (int)ceil_div(pl->tiles_per_unit, 2);
+  pl->ctas = pr.units * pl->pairs_per_unit;
+  const MaskSpec ms{pr.q_len, pr.kv_len, pr.causal, pr.window};
+  int max_tiles = 0;
+  for (int t = 0; t < pl->tiles_per_unit; ++t) {
+    const long long r0 = (long long)t * kPfM;
+    const int nr = (int)((pr.rows - r0) < kPfM ? (pr.rows - r0) : kPfM);
+    const KeyRange kr = key_range(ms, r0, nr, kPfN);
+    if (kr.t_count > max_tiles) max_tiles = kr.t_count;
+  }
+  pl->max_tiles = max_tiles;
+  if (pl->ctas > 0x7fffffffLL) return GQA_ATTN_ERR_TOO_LARGE;
   return GQA_ATTN_OK;
 }
 
@@ -174,40 +203,69 @@ int make_plan(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
     pl->path = kPathZero;
     return GQA_ATTN_OK;
   }
-  return plan_decode(pr, dev, pl);
+  // Short query blocks (<= 64 rows per kv head) are K/V-bandwidth bound: the
+  // split-KV decode kernel.  Longer ones go to the tcgen05 kernel (head_dim
+  // up to 128); the decode kernel also covers head_dim 136..256.
+  const int forced = g_force_path.load();
+  const bool prefill_ok = pr.d <= 128;
+  bool prefill = pr.rows > kDecRows && prefill_ok;
+  if (forced == 1) prefill = false;
+  if (forced == 2 && prefill_ok) prefill = true;
+  return prefill ? plan_prefill(pr, pl) : plan_decode(pr, dev, pl);
 }
 
 // ------------------------------------------------------------------ workspace
 struct Workspace {
   void* ptr = nullptr;
   size_t bytes = 0;
+  void* tickets = nullptr;
+  size_t ticket_bytes = 0;
 };
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
 
-// Workspace of at least `bytes` for (current device, stream).  The ticket
-// region [off_tickets, end) must read as zero: new memory is cleared on the
-// stream; kernels leave their tickets at zero.
-int get_workspace(cudaStream_t stream, size_t bytes, void** out) {
+// Workspace for (current device, stream): `bytes` of scratch for the split
+// partials and `ticket_bytes` of ticket counters.  Tickets live in their own
+// buffer, cleared on allocation; every kernel leaves its tickets at zero.
+int get_workspace(cudaStream_t stream, size_t bytes, size_t ticket_bytes, void** out,
+                  void** tickets) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ATTN_ERR_DEVICE;
   std::lock_guard<std::mutex> lk(g_mu);
   Workspace& ws = g_ws[std::make_pair(dev, stream)];
-  if (ws.bytes < bytes) {
-    if (ws.ptr) {
+  if (ws.bytes < bytes || ws.ticket_bytes < ticket_bytes) {
+    if (ws.ptr || ws.tickets) {
       cudaStreamSynchronize(stream);
-      cudaFree(ws.ptr);
-      ws.ptr = nullptr;
-      ws.bytes = 0;
+      if (ws.bytes < bytes && ws.ptr) {
+        cudaFree(ws.ptr);
+        ws.ptr = nullptr;
+        ws.bytes = 0;
+      }
+      if (ws.ticket_bytes < ticket_bytes && ws.tickets) {
+        cudaFree(ws.tickets);
+        ws.tickets = nullptr;
+        ws.ticket_bytes = 0;
+      }
     }
-    const size_t want = bytes + bytes / 4;
-    if (cudaMalloc(&ws.ptr, want) != cudaSuccess) {
-      cudaGetLastError();
-      return GQA_ATTN_ERR_ALLOC;
+    if (!ws.ptr) {
+      const size_t want = bytes + bytes / 4;
+      if (cudaMalloc(&ws.ptr, want) != cudaSuccess) {
+        cudaGetLastError();
+        return GQA_ATTN_ERR_ALLOC;
+      }
+      ws.bytes = want;
     }
-    if (cudaMemsetAsync(ws.ptr, 0, want, stream) != cudaSuccess) return GQA_ATTN_ERR_LAUNCH;
-    ws.bytes = want;
+    if (!ws.tickets) {
+      const size_t want = ticket_bytes < 4096 ? 4096 : ticket_bytes * 2;
+      if (cudaMalloc(&ws.tickets, want) != cudaSuccess) {
+        cudaGetLastError();
+        return GQA_ATTN_ERR_ALLOC;
+      }
+      if (cudaMemsetAsync(ws.tickets, 0, want, stream) != cudaSuccess) return GQA_ATTN_ERR_LAUNCH;
+      ws.ticket_bytes = want;
+    }
   }
   *out = ws.ptr;
+  *tickets = ws.tickets;
   return GQA_ATTN_OK;
 }
 
@@ -230,7 +288,8 @@ int encode_map(CUtensorMap* map, const void* base, int cols, long long rows, lon
 // ------------------------------------------------------------------ launches
 template <int KS>
 int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
-                     const void* k, const void* v, void* o, void* ws, cudaStream_t stream) {
+                     const void* k, const void* v, void* o, void* ws, void* tickets,
+                     cudaStream_t stream) {
   using C = DecodeCfg<KS>;
   const int slot = KS / 4 - 1;
   if (!dev.decode_attr[slot]) {
@@ -264,20 +323,65 @@ int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.tiles_per_split = pl.tps;
   p.part_o = (float*)ws;
   p.part_lse = ws ? (float*)((char*)ws + pl.off_lse) : nullptr;
-  p.tickets = ws ? (unsigned int*)((char*)ws + pl.off_tickets) : nullptr;
+  p.tickets = (unsigned int*)tickets;
   decode_splitkv_kernel<KS><<<dim3((unsigned)pl.ctas), kDecThreads, C::kSmemBytes, stream>>>(
       tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? GQA_ATTN_OK : GQA_ATTN_ERR_LAUNCH;
 }
 
 int launch_decode(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
-                  const void* k, const void* v, void* o, void* ws, cudaStream_t stream) {
+                  const void* k, const void* v, void* o, void* ws, void* tickets,
+                  cudaStream_t stream) {
   switch (pl.ks) {
-    case 4: return launch_decode_ks<4>(pr, pl, dev, q, k, v, o, ws, stream);
-    case 8: return launch_decode_ks<8>(pr, pl, dev, q, k, v, o, ws, stream);
-    case 12: return launch_decode_ks<12>(pr, pl, dev, q, k, v, o, ws, stream);
-    default: return launch_decode_ks<16>(pr, pl, dev, q, k, v, o, ws, stream);
+    case 4: return launch_decode_ks<4>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+    case 8: return launch_decode_ks<8>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+    case 12: return launch_decode_ks<12>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+    default: return launch_decode_ks<16>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
   }
+}
+
+template <int DCH>
+int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
+                     const void* k, const void* v, void* o, cudaStream_t stream) {
+  using C = PrefillCfg<DCH>;
+  if (!dev.prefill_attr[DCH - 1]) {
+    if (cudaFuncSetAttribute(prefill_sm100_kernel<DCH>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kSmemBytes) != cudaSuccess)
+      return GQA_ATTN_ERR_LAUNCH;
+    dev.prefill_attr[DCH - 1] = true;
+  }
+  CUtensorMap tq, tk, tv;
+  if (encode_map(&tq, q, pr.d, pr.rows, pr.units, kPfM) != GQA_ATTN_OK ||
+      encode_map(&tk, k, pr.d, pr.kv_len, pr.units, kPfN) != GQA_ATTN_OK ||
+      encode_map(&tv, v, pr.d, pr.kv_len, pr.units, kPfN) != GQA_ATTN_OK)
+    return GQA_ATTN_ERR_LAUNCH;
+  PrefillParams p;
+  p.o = (__nv_bfloat16*)o;
+  p.q_len = pr.q_len;
+  p.kv_len = pr.kv_len;
+  p.head_dim = pr.d;
+  p.d_pad = pl.d_pad;
+  p.rows = (int)pr.rows;
+  p.tiles_per_unit = pl.tiles_per_unit;
+  p.pairs_per_unit = pl.pairs_per_unit;
+  p.pair_heads = pl.pair_heads;
+  p.causal = pr.causal;
+  p.window = pr.window;
+  p.use_softcap = pr.softcap > 0.f ? 1 : 0;
+  const float rs = 1.0f / std::sqrt((float)pr.d);
+  p.logit_scale = kLog2e * rs;
+  p.cap_in = p.use_softcap ? rs / pr.softcap : 0.f;
+  p.cap_out = p.use_softcap ? pr.softcap * kLog2e : 0.f;
+  prefill_sm100_kernel<DCH><<<dim3((unsigned)pl.ctas), kPfThreads, C::kSmemBytes, stream>>>(
+      tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? GQA_ATTN_OK : GQA_ATTN_ERR_LAUNCH;
+}
+
+int launch_prefill(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
+                   const void* k, const void* v, void* o, cudaStream_t stream) {
+  return pl.dch == 1 ? launch_prefill_d<1>(pr, pl, dev, q, k, v, o, stream)
+                     : launch_prefill_d<2>(pr, pl, dev, q, k, v, o, stream);
 }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -316,13 +420,16 @@ int run(const Problem& pr, const void* q, const void* k, const void* v, void* o,
       return cudaMemsetAsync(o, 0, bytes, stream) == cudaSuccess ? GQA_ATTN_OK
                                                                  : GQA_ATTN_ERR_LAUNCH;
     }
+    case kPathPrefill:
+      return launch_prefill(pr, pl, *dev, q, k, v, o, stream);
     default: {
       void* ws = nullptr;
+      void* tickets = nullptr;
       if (pl.ws_bytes) {
-        rc = get_workspace(stream, pl.ws_bytes, &ws);
+        rc = get_workspace(stream, pl.ws_bytes, pl.ticket_bytes, &ws, &tickets);
         if (rc != GQA_ATTN_OK) return rc;
       }
-      return launch_decode(pr, pl, *dev, q, k, v, o, ws, stream);
+      return launch_decode(pr, pl, *dev, q, k, v, o, ws, tickets, stream);
     }
   }
 }
