@@ -156,6 +156,13 @@ int gqa_attn_clear_status(void);
  */
 int gqa_attn_selftest_bounded_wait(int limit_us, void* stream);
 
+/*
+ * gqa_attn_last_error_detail -- for the calling thread, which CUDA call
+ * failed last and its error name ("" when none); static thread-local
+ * storage, overwritten by the next failure.
+ */
+const char* gqa_attn_last_error_detail(void);
+
 /* Library version as major * 10000 + minor * 100 + patch. */
 int gqa_attn_version(void);
 

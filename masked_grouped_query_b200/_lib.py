@@ -18,7 +18,7 @@ EXPORTS = (
     "gqa_attn_fwd", "gqa_attn_fwd_host", "gqa_attn_describe",
     "gqa_attn_set_override", "gqa_attn_error_string", "gqa_attn_status",
     "gqa_attn_clear_status", "gqa_attn_selftest_bounded_wait",
-    "gqa_attn_version",
+    "gqa_attn_version", "gqa_attn_last_error_detail",
 )
 
 _I = ctypes.c_int
@@ -35,7 +35,9 @@ class GqaAttnError(RuntimeError):
     """A non-zero return code of the C library."""
 
     def __init__(self, code: int, what: str):
-        super().__init__(f"{what} failed: {error_string(code)} (code {code})")
+        detail = load().gqa_attn_last_error_detail().decode()
+        super().__init__(f"{what} failed: {error_string(code)} (code {code})"
+                         + (f" [{detail}]" if detail else ""))
         self.code = code
 
 
@@ -69,6 +71,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.gqa_attn_selftest_bounded_wait.argtypes = [_I, _P]
         lib.gqa_attn_version.restype = _I
         lib.gqa_attn_version.argtypes = []
+        lib.gqa_attn_last_error_detail.restype = ctypes.c_char_p
+        lib.gqa_attn_last_error_detail.argtypes = []
         if path is None:
             _lib = lib
         return lib

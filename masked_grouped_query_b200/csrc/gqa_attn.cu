@@ -9,6 +9,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -124,6 +125,15 @@ struct Plan {
   size_t off_lse = 0;
   size_t ticket_bytes = 0;  // split tickets (kept zero between calls)
 };
+
+thread_local char g_detail[160] = "";
+
+// Remember which CUDA call failed (readable with gqa_attn_last_error_detail).
+int cuda_fail(const char* where, cudaError_t e, int code) {
+  snprintf(g_detail, sizeof g_detail, "%s: %s (%s)", where, cudaGetErrorName(e),
+           cudaGetErrorString(e));
+  return code;
+}
 
 inline long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -282,7 +292,11 @@ int encode_map(CUtensorMap* map, const void* base, int cols, long long rows, lon
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? GQA_ATTN_OK : GQA_ATTN_ERR_LAUNCH;
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_detail, sizeof g_detail, "cuTensorMapEncodeTiled: CUresult %d", (int)r);
+    return GQA_ATTN_ERR_LAUNCH;
+  }
+  return GQA_ATTN_OK;
 }
 
 // ------------------------------------------------------------------ launches
@@ -293,10 +307,9 @@ int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   using C = DecodeCfg<KS>;
   const int slot = KS / 4 - 1;
   if (!dev.decode_attr[slot]) {
-    if (cudaFuncSetAttribute(decode_splitkv_kernel<KS>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
-      return GQA_ATTN_ERR_LAUNCH;
+    const cudaError_t e = cudaFuncSetAttribute(
+        decode_splitkv_kernel<KS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(decode)", e, GQA_ATTN_ERR_LAUNCH);
     dev.decode_attr[slot] = true;
   }
   CUtensorMap tk, tv;
@@ -326,7 +339,8 @@ int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.tickets = (unsigned int*)tickets;
   decode_splitkv_kernel<KS><<<dim3((unsigned)pl.ctas), kDecThreads, C::kSmemBytes, stream>>>(
       tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? GQA_ATTN_OK : GQA_ATTN_ERR_LAUNCH;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? GQA_ATTN_OK : cuda_fail("launch(decode)", e, GQA_ATTN_ERR_LAUNCH);
 }
 
 int launch_decode(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
@@ -345,10 +359,19 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
                      const void* k, const void* v, void* o, cudaStream_t stream) {
   using C = PrefillCfg<DCH>;
   if (!dev.prefill_attr[DCH - 1]) {
-    if (cudaFuncSetAttribute(prefill_sm100_kernel<DCH>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kSmemBytes) != cudaSuccess)
+    // The register split inside the kernel must fit what the block is
+    // launched with, or setmaxnreg.inc could never be granted.
+    cudaFuncAttributes fa;
+    const cudaError_t ea = cudaFuncGetAttributes(&fa, prefill_sm100_kernel<DCH>);
+    if (ea != cudaSuccess) return cuda_fail("cudaFuncGetAttributes(prefill)", ea, GQA_ATTN_ERR_LAUNCH);
+    if ((long long)fa.numRegs * kPfThreads < kRegSplitTotal) {
+      snprintf(g_detail, sizeof g_detail, "prefill kernel built with %d registers/thread: "
+               "register split needs %d", fa.numRegs, kRegSplitTotal);
       return GQA_ATTN_ERR_LAUNCH;
+    }
+    const cudaError_t e = cudaFuncSetAttribute(
+        prefill_sm100_kernel<DCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(prefill)", e, GQA_ATTN_ERR_LAUNCH);
     dev.prefill_attr[DCH - 1] = true;
   }
   CUtensorMap tq, tk, tv;
@@ -375,7 +398,8 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.cap_out = p.use_softcap ? pr.softcap * kLog2e : 0.f;
   prefill_sm100_kernel<DCH><<<dim3((unsigned)pl.ctas), kPfThreads, C::kSmemBytes, stream>>>(
       tq, tk, tv, p);
-  return cudaGetLastError() == cudaSuccess ? GQA_ATTN_OK : GQA_ATTN_ERR_LAUNCH;
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? GQA_ATTN_OK : cuda_fail("launch(prefill)", e, GQA_ATTN_ERR_LAUNCH);
 }
 
 int launch_prefill(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
@@ -553,5 +577,7 @@ int gqa_attn_selftest_bounded_wait(int limit_us, void* stream) {
 }
 
 int gqa_attn_version(void) { return 100; }
+
+const char* gqa_attn_last_error_detail(void) { return g_detail; }
 
 }  // extern "C"

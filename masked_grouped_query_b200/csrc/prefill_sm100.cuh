@@ -9,7 +9,7 @@
 // feeds both ("north star" (2): the q heads of a GQA group are packed so each
 // K/V tile is read once).
 //
-// Roles (10 warps):
+// Roles (12 warps, three warpgroups):
 //   warp 0      TMA loader: both Q tiles once, then K_j, V_j (128 keys x
 //               head_dim, 128-byte swizzle) into a ring of shared-memory
 //               slots guarded by mbarriers;
@@ -17,7 +17,8 @@
 //               S_t = Q_t K_j^T (M=128, N=128, fp32 in TMEM) and
 //               O_t += P_t V_j (A = P from TMEM, B = V from shared memory,
 //               N = head_dim rounded up to 16);
-//   warps 2-5   softmax + epilogue for tile A, warps 6-9 for tile B: one
+//   warps 2-3   idle (they complete warpgroup 0 for the register split);
+//   warps 4-7   softmax + epilogue for tile A, warps 8-11 for tile B: one
 //               thread per row reads its S row from TMEM, applies scale,
 //               softcap and mask, keeps the running max / sum in fp32
 //               (online softmax, rescaling O in TMEM only when the max grows
@@ -37,8 +38,15 @@ namespace gqa {
 
 constexpr int kPfM = 128;       // rows per q tile
 constexpr int kPfN = 128;       // keys per K/V tile
-constexpr int kPfWarps = 10;
+constexpr int kPfWarps = 12;
 constexpr int kPfThreads = 32 * kPfWarps;
+// Register split (setmaxnreg): the loader/MMA warpgroup drops to kRegsLow,
+// the two softmax warpgroups rise to kRegsHigh.  The host checks before every
+// launch that 4*32*kRegsLow + 8*32*kRegsHigh fits in the registers the block
+// is launched with, so the increase can always be granted.
+constexpr int kRegsLow = 96;
+constexpr int kRegsHigh = 200;
+constexpr int kRegSplitTotal = 4 * 32 * kRegsLow + 8 * 32 * kRegsHigh;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 struct PrefillParams {
@@ -97,7 +105,7 @@ __device__ __forceinline__ TileInfo prefill_tile(const PrefillParams& p, const M
 }
 
 template <int DCH>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kPfThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
@@ -160,9 +168,13 @@ __global__ void __maxnreg__(200)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+
   // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
   // P_t (bf16 pairs) overwrites the first 64 columns of S_t.
 
+  if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
+  }
   if (warp == 0) {
     // ------------------------------------------------------------ loader
     if (lane == 0) {
@@ -281,9 +293,10 @@ __global__ void __maxnreg__(200)
       mma_commit(drain);
       mbar_wait(drain, 0, kStatusTimeoutMma);
     }
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax / epilogue
-    const int t = (warp - 2) / 4;            // tile 0 (A) or 1 (B)
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
+    const int t = (warp - 4) / 4;            // tile 0 (A) or 1 (B)
     const TileInfo& ti = t == 0 ? ta : tb;
     const int quarter = warp & 3;            // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;       // row within the tile
