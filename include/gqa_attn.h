@@ -163,6 +163,38 @@ int gqa_attn_selftest_bounded_wait(int limit_us, void* stream);
  */
 const char* gqa_attn_last_error_detail(void);
 
+/*
+ * gqa_attn_fwd_static_scratch -- gqa_attn_fwd for callers that cannot
+ * allocate device memory, restricted to the split-KV decode kernel.
+ *
+ * The pages describe no such entry point; it exists for callers who may not
+ * call cudaMalloc: code whose device memory is all handed to its own pool
+ * (an allocation outside the pool fails or fragments it), and latency-bound
+ * callers that cannot take the device-wide synchronisation cudaMalloc and
+ * cudaFree can cause.  gqa_attn_fwd allocates its split workspace on first
+ * need; this variant allocates nothing and calls no allocating routine.
+ *
+ * Arguments, layouts, ownership and return codes are those of gqa_attn_fwd;
+ * the computation is always the split-KV decode kernel (any sizes it takes,
+ * head_dim up to 256).  Its scratch (split partials and tickets) is one
+ * file-scope device array of 8 MiB (64 KiB of tickets + 8128 KiB of
+ * partials) that every GPU loading this library holds until the process
+ * exits.  A plan whose partials or tickets exceed it returns
+ * GQA_ATTN_ERR_TOO_LARGE (see gqa_attn_last_error_detail); plans with one
+ * split use no scratch.  Each call clears the tickets it uses with
+ * cudaMemsetAsync on `stream` before the kernel.
+ *
+ * The first call on a device looks the array's device address up
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  All calls share the one array: calls whose
+ * execution overlaps on the GPU (other streams, other threads) race on it,
+ * so serialise them.
+ */
+int gqa_attn_fwd_static_scratch(const void* q, const void* k, const void* v, void* o, int batch,
+                                int q_len, int kv_len, int num_q_heads, int num_kv_heads,
+                                int head_dim, int causal, int window, float softcap,
+                                void* stream);
+
 /* Library version as major * 10000 + minor * 100 + patch. */
 int gqa_attn_version(void);
 

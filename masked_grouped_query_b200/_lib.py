@@ -18,7 +18,7 @@ EXPORTS = (
     "gqa_attn_fwd", "gqa_attn_fwd_host", "gqa_attn_describe",
     "gqa_attn_set_override", "gqa_attn_error_string", "gqa_attn_status",
     "gqa_attn_clear_status", "gqa_attn_selftest_bounded_wait",
-    "gqa_attn_version", "gqa_attn_last_error_detail",
+    "gqa_attn_version", "gqa_attn_last_error_detail", "gqa_attn_fwd_static_scratch",
 )
 
 _I = ctypes.c_int
@@ -73,6 +73,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.gqa_attn_version.argtypes = []
         lib.gqa_attn_last_error_detail.restype = ctypes.c_char_p
         lib.gqa_attn_last_error_detail.argtypes = []
+        lib.gqa_attn_fwd_static_scratch.restype = _I
+        lib.gqa_attn_fwd_static_scratch.argtypes = [_P, _P, _P, _P] + _DIMS + [_P]
         if path is None:
             _lib = lib
         return lib

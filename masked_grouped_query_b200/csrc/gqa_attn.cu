@@ -458,6 +458,36 @@ int run(const Problem& pr, const void* q, const void* k, const void* v, void* o,
   }
 }
 
+// ------------------------------------------------------------------ static scratch
+// Scratch for gqa_attn_fwd_static_scratch: a fixed array in device memory,
+// created with the module on every GPU that loads this library and kept
+// until the process exits.  Layout: [0, kStaticTicketBytes) split tickets,
+// then the split partials (o_s, then lse_s).  Host code must not pass the
+// array's name to a kernel (in host code it is only a stand-in for the
+// symbol); its device address comes from cudaGetSymbolAddress below.
+constexpr size_t kStaticScratchBytes = 8u << 20;  // 8 MiB
+constexpr size_t kStaticTicketBytes = 64u << 10;  // 16384 tickets
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+void* g_static_scratch_addr[64] = {};
+
+// Device address of g_static_scratch on the current device, looked up once
+// per device (with that device current) and cached.
+int static_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return GQA_ATTN_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_static_scratch_addr[dev]) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_static_scratch);
+    if (e != cudaSuccess || ptr == nullptr)
+      return cuda_fail("cudaGetSymbolAddress(g_static_scratch)", e, GQA_ATTN_ERR_LAUNCH);
+    g_static_scratch_addr[dev] = ptr;
+  }
+  *out = g_static_scratch_addr[dev];
+  return GQA_ATTN_OK;
+}
+
 }  // namespace
 
 // ==================================================================== C ABI
@@ -579,5 +609,46 @@ int gqa_attn_selftest_bounded_wait(int limit_us, void* stream) {
 int gqa_attn_version(void) { return 100; }
 
 const char* gqa_attn_last_error_detail(void) { return g_detail; }
+
+int gqa_attn_fwd_static_scratch(const void* q, const void* k, const void* v, void* o, int batch,
+                                int q_len, int kv_len, int num_q_heads, int num_kv_heads,
+                                int head_dim, int causal, int window, float softcap,
+                                void* stream) {
+  Problem pr;
+  int rc = validate(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, causal, window,
+                    softcap, &pr);
+  if (rc != GQA_ATTN_OK) return rc;
+  rc = check_pointers(pr, q, k, v, o);
+  if (rc != GQA_ATTN_OK) return rc;
+  DeviceInfo* dev = nullptr;
+  rc = device_info(&dev);
+  if (rc != GQA_ATTN_OK) return rc;
+  void* scratch = nullptr;
+  rc = static_scratch(&scratch);  // first call on a device: symbol lookup
+  if (rc != GQA_ATTN_OK) return rc;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (pr.batch == 0 || pr.q_len == 0) return GQA_ATTN_OK;
+  if (pr.kv_len == 0) {
+    const size_t bytes = (size_t)pr.batch * pr.hq * (size_t)pr.q_len * pr.d * 2;
+    const cudaError_t e = cudaMemsetAsync(o, 0, bytes, s);
+    return e == cudaSuccess ? GQA_ATTN_OK : cuda_fail("cudaMemsetAsync(o)", e, GQA_ATTN_ERR_LAUNCH);
+  }
+  Plan pl;
+  rc = plan_decode(pr, *dev, &pl);
+  if (rc != GQA_ATTN_OK) return rc;
+  if (pl.splits == 1) return launch_decode(pr, pl, *dev, q, k, v, o, nullptr, nullptr, s);
+  if (pl.ticket_bytes > kStaticTicketBytes ||
+      pl.ws_bytes > kStaticScratchBytes - kStaticTicketBytes) {
+    snprintf(g_detail, sizeof g_detail,
+             "static scratch too small: needs %zu bytes of partials and %zu of tickets, "
+             "has %zu and %zu", pl.ws_bytes, pl.ticket_bytes,
+             kStaticScratchBytes - kStaticTicketBytes, kStaticTicketBytes);
+    return GQA_ATTN_ERR_TOO_LARGE;
+  }
+  // Tickets must start at zero; the array keeps whatever the last call left.
+  const cudaError_t e = cudaMemsetAsync(scratch, 0, pl.ticket_bytes, s);
+  if (e != cudaSuccess) return cuda_fail("cudaMemsetAsync(tickets)", e, GQA_ATTN_ERR_LAUNCH);
+  return launch_decode(pr, pl, *dev, q, k, v, o, (char*)scratch + kStaticTicketBytes, scratch, s);
+}
 
 }  // extern "C"
