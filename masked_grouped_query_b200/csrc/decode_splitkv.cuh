@@ -64,8 +64,14 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
-template <int KS>
-__global__ void __launch_bounds__(kDecThreads, 1)
+// kT = true: the variant for row blocks of at most 8 rows (single-token GQA
+// decode).  Keys become the M dimension of the tensor-core tiles --
+// S^T = K Q^T (m16 keys x n8 rows) and O^T += V^T P^T (m16 head-dim x n8
+// rows), with P^T moved into the B-operand layout by movmatrix -- so the
+// padded rows cost half as much as in the rows-as-M form and the O
+// accumulator needs half the registers (two CTAs per SM).
+template <int KS, bool kT>
+__global__ void __maxnreg__(kT ? 128 : 255)
     decode_splitkv_kernel(const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
   using C = DecodeCfg<KS>;
@@ -132,11 +138,139 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
 
   // -------------------------------------------------------------- compute
-  const int wm_count = nr <= 16 ? 1 : (nr <= 32 ? 2 : 4);
+  const int wm_count = kT ? 1 : (nr <= 16 ? 1 : (nr <= 32 ? 2 : 4));
   const int wn_count = kDecComputeWarps / wm_count;
+  const int D = p.head_dim;
+  const int DP = KS * 16;  // padded head dim
+  float* mrg = (float*)smem;
+  if constexpr (kT) {
+    const int wn = warp;  // 16 keys of every 64-key tile
+    const int g = lane >> 2, t4 = lane & 3;
+    // Q^T fragments (B operand: k = head dim, n = row), straight from global.
+    uint32_t qb[KS][2];
+    {
+      const __nv_bfloat16* qrow = p.q + ((long long)unit * p.rows + r0 + g) * D;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int d = ks * 16 + h * 8 + 2 * t4;
+          qb[ks][h] = (g < nr && d < D) ? *(const uint32_t*)(qrow + d) : 0u;
+        }
+    }
+    int lo[2], hi[2];  // rows 2*t4 and 2*t4 + 1
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const long long r = r0 + 2 * t4 + h;
+      const int qpos = p.kv_len - p.q_len + (int)(r % p.q_len);
+      lo[h] = first_key(ms, qpos);
+      hi[h] = last_key(ms, qpos);
+    }
+    float ot[KS][4];
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) ot[mt][0] = ot[mt][1] = ot[mt][2] = ot[mt][3] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+    const int mi = lane >> 3, rr = lane & 7;
+    for (int t = 0; t < n_tiles; ++t) {
+      const int s = t % C::kStages;
+      if (!mbar_wait(&full[s], (t / C::kStages) & 1, kStatusTimeoutConsumer)) break;
+      const uint32_t kbase = smem_u32(ring + s * C::kStageBytes);
+      const uint32_t vbase = kbase + C::kTileBytes;
+      const int key0 = (kr.t_first + t_begin + t) * kDecTile;
+      const int wkey0 = wn * 16;
+      const bool need_mask = !(key0 >= kr.all_lo && key0 + kDecTile - 1 <= kr.all_hi);
+      // ---- S^T = K Q^T (16 keys x 8 rows)
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int key = wkey0 + (mi & 1) * 8 + rr;
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(kbase + (ks >> 2) * C::kBoxBytes + sw128(key, (ks * 2 + (mi >> 1)) & 7), a0, a1,
+                  a2, a3);
+          mma_16816(sc, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+        }
+      }
+      // ---- logits: element e is (key g + 8*(e>>1), row 2*t4 + (e&1))
+      float x[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float v = p.use_softcap ? p.cap_out * tanh_accurate(sc[e] * p.cap_in) : sc[e] * p.logit_scale;
+        if (need_mask) {
+          const int j = key0 + wkey0 + g + 8 * (e >> 1);
+          if (j < lo[e & 1] || j > hi[e & 1]) v = -INFINITY;
+        }
+        x[e] = v;
+      }
+      float base[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float m = fmaxf(x[h], x[h + 2]);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        const float m_new = fmaxf(m_run[h], m);
+        // Rescale only when the max grew by more than 2^8 (or was -inf).
+        if (m_new > m_run[h] + 8.0f || (m_run[h] == -INFINITY && m_new != -INFINITY)) {
+          const float alpha = ex2(m_run[h] - m_new);
+          m_run[h] = m_new;
+          l_run[h] *= alpha;
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            ot[mt][h] *= alpha;
+            ot[mt][h + 2] *= alpha;
+          }
+        }
+        base[h] = m_run[h] == -INFINITY ? 0.f : m_run[h];
+      }
+      float pr[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        pr[e] = ex2(x[e] - base[e & 1]);
+        l_run[e & 1] += pr[e];
+      }
+      const uint32_t b0 = movmatrix_t(pack_bf16(pr[0], pr[1]));
+      const uint32_t b1 = movmatrix_t(pack_bf16(pr[2], pr[3]));
+      // ---- O^T += V^T P^T (head dim 16 at a time)
+      {
+        const int key = wkey0 + (mi >> 1) * 8 + rr;
+#pragma unroll
+        for (int mt = 0; mt < KS; ++mt) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(vbase + (mt >> 2) * C::kBoxBytes + sw128(key, (mt * 2 + (mi & 1)) & 7), a0,
+                    a1, a2, a3);
+          mma_16816(ot[mt], a0, a1, a2, a3, b0, b1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    // l is a per-thread partial over its keys: reduce over the 8 lanes of a row.
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 4);
+      l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 8);
+      l_run[h] += __shfl_xor_sync(0xffffffffu, l_run[h], 16);
+    }
+    __syncthreads();  // (A) ring drained and no longer read: reuse it as merge scratch
+    float* so = mrg + wn * 16 * (DP + 2);
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float* row = so + (2 * t4 + h) * (DP + 2);
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        row[mt * 16 + g] = ot[mt][h];
+        row[mt * 16 + g + 8] = ot[mt][h + 2];
+      }
+      if (g == 0) {
+        row[DP] = m_run[h];
+        row[DP + 1] = l_run[h];
+      }
+    }
+  } else {
   const int wm = warp % wm_count, wn = warp / wm_count;
   const int kw = kDecTile / wn_count;  // keys per warp per tile: 64, 32 or 16
-  const int D = p.head_dim;
   const int g_row_base = wm * 16 + (lane >> 2);  // CTA row of c0/c1; +8 for c2/c3
 
   // Q fragments (A operand, row-major 16 x 16 per k-step), straight from global.
@@ -279,8 +413,6 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 
   // ---- merge the key-slices of the warps through shared memory
   __syncthreads();  // (A) ring drained and no longer read: reuse it as merge scratch
-  const int DP = KS * 16;  // padded head dim
-  float* mrg = (float*)smem;
   {
     const int slot = wn * wm_count + wm;  // 0..3
     float* so = mrg + slot * 16 * (DP + 2);
@@ -298,6 +430,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         row[DP + 1] = l_run[h];
       }
     }
+  }
   }
   asm volatile("bar.sync 1, %0;" ::"r"(kDecComputeWarps * 32) : "memory");
 

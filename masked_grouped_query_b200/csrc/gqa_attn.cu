@@ -34,7 +34,7 @@ struct DeviceInfo {
   bool probed = false;
   int sms = 0, major = 0, minor = 0;
   int smem_optin = 0;
-  bool decode_attr[4] = {false, false, false, false};
+  bool decode_attr[8] = {false, false, false, false, false, false, false, false};
   bool prefill_attr[2] = {false, false};
 };
 
@@ -160,8 +160,14 @@ int plan_decode(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
   } else if (forced > 0) {
     tps = forced;
   } else {
-    const long long want = ceil_div(8LL * dev.sms, base);
-    tps = (int)ceil_div(max_tiles, want < 1 ? 1 : want);
+    // Splits per row block, measured on B200 (L2 flushed): single-token
+    // blocks (keys-as-M variant, two CTAs per SM) do best with ~3.5 CTAs per
+    // SM in total; larger row blocks (one CTA per SM, partial traffic of 64
+    // rows per split) with about two thirds of a wave.
+    const double per_sm = pl->block_rows <= 8 ? 3.5 : 0.65;
+    long long want = (long long)(per_sm * dev.sms / (double)base + 0.5);
+    if (want < 1) want = 1;
+    tps = (int)ceil_div(max_tiles, want);
     if (tps < 4) tps = 4;
   }
   if (tps > max_tiles && max_tiles > 0) tps = max_tiles;
@@ -300,15 +306,20 @@ int encode_map(CUtensorMap* map, const void* base, int cols, long long rows, lon
 }
 
 // ------------------------------------------------------------------ launches
-template <int KS>
+template <int KS, bool kT>
 int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
                      const void* k, const void* v, void* o, void* ws, void* tickets,
                      cudaStream_t stream) {
   using C = DecodeCfg<KS>;
-  const int slot = KS / 4 - 1;
+  const int slot = (KS / 4 - 1) + (kT ? 4 : 0);
   if (!dev.decode_attr[slot]) {
-    const cudaError_t e = cudaFuncSetAttribute(
-        decode_splitkv_kernel<KS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(decode_splitkv_kernel<KS, kT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_splitkv_kernel<KS, kT>,
+                               cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(decode)", e, GQA_ATTN_ERR_LAUNCH);
     dev.decode_attr[slot] = true;
   }
@@ -337,8 +348,8 @@ int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.part_o = (float*)ws;
   p.part_lse = ws ? (float*)((char*)ws + pl.off_lse) : nullptr;
   p.tickets = (unsigned int*)tickets;
-  decode_splitkv_kernel<KS><<<dim3((unsigned)pl.ctas), kDecThreads, C::kSmemBytes, stream>>>(
-      tk, tv, p);
+  decode_splitkv_kernel<KS, kT>
+      <<<dim3((unsigned)pl.ctas), kDecThreads, C::kSmemBytes, stream>>>(tk, tv, p);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? GQA_ATTN_OK : cuda_fail("launch(decode)", e, GQA_ATTN_ERR_LAUNCH);
 }
@@ -346,11 +357,19 @@ int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
 int launch_decode(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
                   const void* k, const void* v, void* o, void* ws, void* tickets,
                   cudaStream_t stream) {
+  if (pl.block_rows <= 8) {  // single-token decode shapes: keys-as-M variant
+    switch (pl.ks) {
+      case 4: return launch_decode_ks<4, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+      case 8: return launch_decode_ks<8, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+      case 12: return launch_decode_ks<12, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+      default: return launch_decode_ks<16, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+    }
+  }
   switch (pl.ks) {
-    case 4: return launch_decode_ks<4>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
-    case 8: return launch_decode_ks<8>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
-    case 12: return launch_decode_ks<12>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
-    default: return launch_decode_ks<16>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+    case 4: return launch_decode_ks<4, false>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+    case 8: return launch_decode_ks<8, false>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+    case 12: return launch_decode_ks<12, false>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+    default: return launch_decode_ks<16, false>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
   }
 }
 
