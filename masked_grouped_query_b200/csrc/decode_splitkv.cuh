@@ -59,11 +59,6 @@ struct DecodeCfg {
       1024 + (kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes) + 2 * kStages * 8 + 64;
 };
 
-// Byte offset of (row, 8-column chunk) inside a 128B-swizzled 64-column box.
-__device__ __forceinline__ uint32_t sw128(int row, int chunk) {
-  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
-}
-
 // kT = true: the variant for row blocks of at most 8 rows (single-token GQA
 // decode).  Keys become the M dimension of the tensor-core tiles --
 // S^T = K Q^T (m16 keys x n8 rows) and O^T += V^T P^T (m16 head-dim x n8

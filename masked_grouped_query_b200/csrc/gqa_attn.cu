@@ -35,7 +35,7 @@ struct DeviceInfo {
   int sms = 0, major = 0, minor = 0;
   int smem_optin = 0;
   bool decode_attr[8] = {false, false, false, false, false, false, false, false};
-  bool prefill_attr[2] = {false, false};
+  bool prefill_attr[4] = {false, false, false, false};
 };
 
 std::mutex g_mu;
@@ -373,15 +373,15 @@ int launch_decode(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void
   }
 }
 
-template <int DCH>
+template <int DCH, bool kCap>
 int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
                      const void* k, const void* v, void* o, cudaStream_t stream) {
   using C = PrefillCfg<DCH>;
-  if (!dev.prefill_attr[DCH - 1]) {
+  if (!dev.prefill_attr[(DCH - 1) + (kCap ? 2 : 0)]) {
     // The register split inside the kernel must fit what the block is
     // launched with, or setmaxnreg.inc could never be granted.
     cudaFuncAttributes fa;
-    const cudaError_t ea = cudaFuncGetAttributes(&fa, prefill_sm100_kernel<DCH>);
+    const cudaError_t ea = cudaFuncGetAttributes(&fa, prefill_sm100_kernel<DCH, kCap>);
     if (ea != cudaSuccess) return cuda_fail("cudaFuncGetAttributes(prefill)", ea, GQA_ATTN_ERR_LAUNCH);
     if ((long long)fa.numRegs * kPfThreads < kRegSplitTotal) {
       snprintf(g_detail, sizeof g_detail, "prefill kernel built with %d registers/thread: "
@@ -389,12 +389,13 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
       return GQA_ATTN_ERR_LAUNCH;
     }
     const cudaError_t e = cudaFuncSetAttribute(
-        prefill_sm100_kernel<DCH>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        prefill_sm100_kernel<DCH, kCap>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(prefill)", e, GQA_ATTN_ERR_LAUNCH);
-    dev.prefill_attr[DCH - 1] = true;
+    dev.prefill_attr[(DCH - 1) + (kCap ? 2 : 0)] = true;
   }
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, to;
   if (encode_map(&tq, q, pr.d, pr.rows, pr.units, kPfM) != GQA_ATTN_OK ||
+      encode_map(&to, o, pr.d, pr.rows, pr.units, 32) != GQA_ATTN_OK ||
       encode_map(&tk, k, pr.d, pr.kv_len, pr.units, kPfN) != GQA_ATTN_OK ||
       encode_map(&tv, v, pr.d, pr.kv_len, pr.units, kPfN) != GQA_ATTN_OK)
     return GQA_ATTN_ERR_LAUNCH;
@@ -407,24 +408,29 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.rows = (int)pr.rows;
   p.tiles_per_unit = pl.tiles_per_unit;
   p.pairs_per_unit = pl.pairs_per_unit;
+  p.n_items = (int)pl.ctas;
   p.pair_heads = pl.pair_heads;
   p.causal = pr.causal;
   p.window = pr.window;
-  p.use_softcap = pr.softcap > 0.f ? 1 : 0;
   const float rs = 1.0f / std::sqrt((float)pr.d);
   p.logit_scale = kLog2e * rs;
-  p.cap_in = p.use_softcap ? rs / pr.softcap : 0.f;
-  p.cap_out = p.use_softcap ? pr.softcap * kLog2e : 0.f;
-  prefill_sm100_kernel<DCH><<<dim3((unsigned)pl.ctas), kPfThreads, C::kSmemBytes, stream>>>(
-      tq, tk, tv, p);
+  p.cap_in = kCap ? rs / pr.softcap : 0.f;
+  p.cap_out = kCap ? pr.softcap * kLog2e : 0.f;
+  // Persistent: at most one CTA per SM, each walking items with stride grid.
+  const int grid = (int)(pl.ctas < dev.sms ? pl.ctas : dev.sms);
+  prefill_sm100_kernel<DCH, kCap><<<dim3((unsigned)grid), kPfThreads, C::kSmemBytes, stream>>>(
+      tq, tk, tv, to, p);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? GQA_ATTN_OK : cuda_fail("launch(prefill)", e, GQA_ATTN_ERR_LAUNCH);
 }
 
 int launch_prefill(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
                    const void* k, const void* v, void* o, cudaStream_t stream) {
-  return pl.dch == 1 ? launch_prefill_d<1>(pr, pl, dev, q, k, v, o, stream)
-                     : launch_prefill_d<2>(pr, pl, dev, q, k, v, o, stream);
+  if (pr.softcap > 0.f)
+    return pl.dch == 1 ? launch_prefill_d<1, true>(pr, pl, dev, q, k, v, o, stream)
+                       : launch_prefill_d<2, true>(pr, pl, dev, q, k, v, o, stream);
+  return pl.dch == 1 ? launch_prefill_d<1, false>(pr, pl, dev, q, k, v, o, stream)
+                     : launch_prefill_d<2, false>(pr, pl, dev, q, k, v, o, stream);
 }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {

@@ -3,16 +3,21 @@
 //
 // Rows: for one (batch b, kv head) unit, the R = group * q_len q rows of all
 // q heads of the GQA group, in memory order (head-major, then position), are
-// cut into 128-row tiles.  A CTA owns two tiles whose key ranges coincide or
-// overlap (two heads of the group at the same positions when q_len is a
-// multiple of 128, else two consecutive tiles), so every K/V tile it loads
-// feeds both ("north star" (2): the q heads of a GQA group are packed so each
-// K/V tile is read once).
+// cut into 128-row tiles.  A work item is a pair of tiles whose key ranges
+// coincide or overlap (two heads of the group at the same positions when
+// q_len is a multiple of 128, else two consecutive tiles), so every K/V tile
+// loaded for the item feeds both ("north star" (2): the q heads of a GQA
+// group are packed so each K/V tile is read once).
+//
+// Persistent: one CTA per SM walks the items blockIdx.x, blockIdx.x +
+// gridDim.x, ...; TMEM, barriers and the K/V ring live across items, and the
+// next item's Q is loaded as soon as the current item's last S = Q K^T has
+// been computed, so loads, MMAs and softmax of consecutive items overlap.
 //
 // Roles (12 warps, three warpgroups):
-//   warp 0      TMA loader: both Q tiles once, then K_j, V_j (128 keys x
-//               head_dim, 128-byte swizzle) into a ring of shared-memory
-//               slots guarded by mbarriers;
+//   warp 0      TMA loader: Q tiles, then K_j, V_j (128 keys x head_dim,
+//               128-byte swizzle) into a ring of shared-memory slots guarded
+//               by mbarriers;
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
 //               S_t = Q_t K_j^T (M=128, N=128, fp32 in TMEM) and
 //               O_t += P_t V_j (A = P from TMEM, B = V from shared memory,
@@ -23,9 +28,10 @@
 //               softcap and mask, keeps the running max / sum in fp32
 //               (online softmax, rescaling O in TMEM only when the max grows
 //               by more than 2^8), writes P as bf16 back over S in TMEM, and
-//               at the end normalises O and stores bf16 rows of o.
-// The issue order S_A(j+1) after PV_A(j), S_B(j+1) after PV_B(j) keeps the
-// tensor pipe busy with one tile while the other tile's softmax runs.
+//               at the end of the item normalises O and stores its bf16 row.
+// Tile B's first S is issued only once tile A's first P is ready, so the two
+// softmax warpgroups run out of phase: while one computes its softmax the
+// tensor core works on the other tile's P.V and next S.
 //
 // Fully masked key tiles are never loaded; tiles wholly inside every row's
 // visible range skip the per-element mask.  All waits are bounded.
@@ -54,10 +60,10 @@ struct PrefillParams {
   int q_len, kv_len, head_dim, d_pad;
   int rows;              // rows per unit: group * q_len
   int tiles_per_unit;    // ceil(rows / 128)
-  int pairs_per_unit;    // CTAs per unit
+  int pairs_per_unit;    // work items per unit
+  int n_items;           // units * pairs_per_unit
   int pair_heads;        // 1: tiles (2p, 2p+1) are two heads at one position
   int causal, window;
-  int use_softcap;
   float logit_scale, cap_in, cap_out;
 };
 
@@ -68,9 +74,11 @@ struct PrefillCfg {
   static constexpr int kSlots = DCH == 1 ? 8 : 4;
   static constexpr int kQBytes = 2 * kTileBytes;
   static constexpr int kRingBytes = kSlots * kTileBytes;
-  static constexpr int kBarOffset = kQBytes + kRingBytes;
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain
-  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 2 + 1;
+  // Output staging: one 32-row x 64-column bf16 box (4 KB) per softmax warp.
+  static constexpr int kStageBytes = 8 * 4096;
+  static constexpr int kBarOffset = kQBytes + kRingBytes + kStageBytes;
+  // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain
+  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 1;
   static constexpr int kSmemBytes = 1024 + kBarOffset + kNumBars * 8 + 16;
 };
 
@@ -104,19 +112,61 @@ __device__ __forceinline__ TileInfo prefill_tile(const PrefillParams& p, const M
   return ti;
 }
 
-template <int DCH>
+// One work item: a unit and its pair of q tiles, with the union of their
+// key-tile ranges [j_first, j_first + j_count).  An item without key tiles
+// is not "busy": its rows (if any) are written as zeros without MMAs.
+struct PfItem {
+  int unit;
+  TileInfo tile[2];
+  int j_first, j_count;
+  bool busy;
+};
+
+__device__ __forceinline__ PfItem prefill_item(const PrefillParams& p, const MaskSpec& ms,
+                                               int item) {
+  PfItem it;
+  it.unit = item / p.pairs_per_unit;
+  const int pair = item % p.pairs_per_unit;
+  it.tile[0] = prefill_tile(p, ms, pair, 0);
+  it.tile[1] = prefill_tile(p, ms, pair, 1);
+  const KeyRange& a = it.tile[0].kr;
+  const KeyRange& b = it.tile[1].kr;
+  if (a.t_count == 0 && b.t_count == 0) {
+    it.j_first = 0;
+    it.j_count = 0;
+  } else {
+    const int fa = a.t_count ? a.t_first : 0x7fffffff, fb = b.t_count ? b.t_first : 0x7fffffff;
+    const int la = a.t_count ? a.t_first + a.t_count - 1 : -1;
+    const int lb = b.t_count ? b.t_first + b.t_count - 1 : -1;
+    it.j_first = min(fa, fb);
+    it.j_count = max(la, lb) - it.j_first + 1;
+  }
+  it.busy = it.j_count > 0;
+  return it;
+}
+
+__device__ __forceinline__ bool tile_active(const PfItem& it, int t, int j) {
+  const KeyRange& kr = t == 0 ? it.tile[0].kr : it.tile[1].kr;
+  const int jj = it.j_first + j;
+  return kr.t_count > 0 && jj >= kr.t_first && jj < kr.t_first + kr.t_count;
+}
+
+template <int DCH, bool kCap>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
-                         const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+                         const __grid_constant__ CUtensorMap tm_v,
+                         const __grid_constant__ CUtensorMap tm_o, const PrefillParams p) {
   using C = PrefillCfg<DCH>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sq = smem;                   // Q tiles A, B
   uint8_t* ring = smem + C::kQBytes;    // K/V slots
+  uint8_t* stage_all = ring + C::kRingBytes;  // output staging, 4 KB per softmax warp
   uint64_t* bars = (uint64_t*)(smem + C::kBarOffset);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;
   uint64_t* kv_empty = kv_full + C::kSlots;
   uint64_t* s_full = kv_empty + C::kSlots;
   uint64_t* p_full = s_full + 2;
@@ -125,29 +175,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint32_t* tmem_slot = (uint32_t*)(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int unit = blockIdx.x / p.pairs_per_unit;
-  const int pair = blockIdx.x % p.pairs_per_unit;
   const MaskSpec ms{p.q_len, p.kv_len, p.causal, p.window};
-  const TileInfo ta = prefill_tile(p, ms, pair, 0);
-  const TileInfo tb = prefill_tile(p, ms, pair, 1);
-  // Key tiles of the CTA: the union of both tiles' ranges.
-  int j_first, j_count;
-  {
-    const bool ea = ta.kr.t_count == 0, eb = tb.kr.t_count == 0;
-    if (ea && eb) {
-      j_first = 0;
-      j_count = 0;
-    } else {
-      const int fa = ea ? 0x7fffffff : ta.kr.t_first, fb = eb ? 0x7fffffff : tb.kr.t_first;
-      const int la = ea ? -1 : ta.kr.t_first + ta.kr.t_count - 1;
-      const int lb = eb ? -1 : tb.kr.t_first + tb.kr.t_count - 1;
-      j_first = min(fa, fb);
-      j_count = max(la, lb) - j_first + 1;
-    }
-  }
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < C::kSlots; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
@@ -168,7 +200,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
   // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
   // P_t (bf16 pairs) overwrites the first 64 columns of S_t.
 
@@ -181,114 +212,136 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
-      const int nq = (ta.nrows > 0 ? 1 : 0) + (tb.nrows > 0 ? 1 : 0);
-      if (nq > 0 && j_count > 0) {
-        mbar_arrive_expect_tx(q_full, nq * C::kTileBytes);
-        for (int c = 0; c < DCH; ++c) {
-          if (ta.nrows > 0)
-            tma_load_3d(sq + c * C::kBoxBytes, &tm_q, q_full, c * 64, ta.row0, unit);
-          if (tb.nrows > 0)
-            tma_load_3d(sq + C::kTileBytes + c * C::kBoxBytes, &tm_q, q_full, c * 64, tb.row0,
-                        unit);
-        }
-      }
-      int issued = 0;
+      int u = 0;       // K/V tiles issued (ring position)
+      int nq = 0;      // busy items whose Q was issued
       bool ok = true;
-      for (int j = 0; j < j_count && ok; ++j) {
-        const int key0 = (j_first + j) * kPfN;
-        for (int kv = 0; kv < 2; ++kv) {
-          const int u = 2 * j + kv;
-          const int s = u % C::kSlots;
-          if (u >= C::kSlots &&
-              !mbar_wait(&kv_empty[s], ((u / C::kSlots) - 1) & 1, kStatusTimeoutProducer)) {
-            ok = false;
-            break;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const PfItem it = prefill_item(p, ms, item);
+        if (!it.busy) continue;
+        // The Q buffer is free once every S of the previous busy item is done.
+        if (nq > 0 && !(ok = mbar_wait(q_empty, (nq - 1) & 1, kStatusTimeoutProducer))) break;
+        const int ntiles = (it.tile[0].nrows > 0 ? 1 : 0) + (it.tile[1].nrows > 0 ? 1 : 0);
+        mbar_arrive_expect_tx(q_full, ntiles * C::kTileBytes);
+        for (int t = 0; t < 2; ++t)
+          if (it.tile[t].nrows > 0)
+            for (int c = 0; c < DCH; ++c)
+              tma_load_3d(sq + t * C::kTileBytes + c * C::kBoxBytes, &tm_q, q_full, c * 64,
+                          it.tile[t].row0, it.unit);
+        ++nq;
+        for (int j = 0; j < it.j_count && ok; ++j) {
+          const int key0 = (it.j_first + j) * kPfN;
+          for (int kv = 0; kv < 2; ++kv) {
+            const int s = u % C::kSlots;
+            if (u >= C::kSlots &&
+                !(ok = mbar_wait(&kv_empty[s], ((u / C::kSlots) - 1) & 1,
+                                 kStatusTimeoutProducer)))
+              break;
+            uint8_t* dst = ring + s * C::kTileBytes;
+            mbar_arrive_expect_tx(&kv_full[s], C::kTileBytes);
+            for (int c = 0; c < DCH; ++c)
+              tma_load_3d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, &kv_full[s], c * 64, key0,
+                          it.unit);
+            ++u;
           }
-          uint8_t* dst = ring + s * C::kTileBytes;
-          mbar_arrive_expect_tx(&kv_full[s], C::kTileBytes);
-          for (int c = 0; c < DCH; ++c)
-            tma_load_3d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, &kv_full[s], c * 64, key0,
-                        unit);
-          ++issued;
         }
       }
       // Drain: never leave with copies in flight.
-      if (nq > 0 && j_count > 0) mbar_wait(q_full, 0, kStatusTimeoutProducer);
-      for (int u = max(0, issued - C::kSlots); u < issued; ++u)
-        mbar_wait(&kv_full[u % C::kSlots], (u / C::kSlots) & 1, kStatusTimeoutProducer);
+      if (nq > 0) mbar_wait(q_full, (nq - 1) & 1, kStatusTimeoutProducer);
+      for (int v = max(0, u - C::kSlots); v < u; ++v)
+        mbar_wait(&kv_full[v % C::kSlots], (v / C::kSlots) & 1, kStatusTimeoutProducer);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && j_count > 0) {
+    if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kPfM, kPfN, 0);
       const uint32_t idesc_o = idesc_bf16_f32(kPfM, p.d_pad, 1);
       const int ksteps = p.d_pad / 16;
       const uint32_t sq_addr = smem_u32(sq);
       const uint32_t ring_addr = smem_u32(ring);
-      int n_act[2] = {0, 0};
-      bool ok = mbar_wait(q_full, 0, kStatusTimeoutMma);
-
-      auto active = [&](int t, int j) {
-        const KeyRange& kr = t == 0 ? ta.kr : tb.kr;
-        const int jj = j_first + j;
-        return kr.t_count > 0 && jj >= kr.t_first && jj < kr.t_first + kr.t_count;
-      };
-      auto wait_slot = [&](int u) {
-        return mbar_wait(&kv_full[u % C::kSlots], (u / C::kSlots) & 1, kStatusTimeoutMma);
-      };
-      auto issue_s = [&](int t, int j) {
-        const uint32_t kslot = ring_addr + ((2 * j) % C::kSlots) * C::kTileBytes;
-        const uint32_t qt = sq_addr + t * C::kTileBytes;
-        const uint32_t d_tmem = tmem + t * 128;
-        tc_fence_after();
-        for (int ks = 0; ks < ksteps; ++ks) {
-          const uint32_t off = (ks >> 2) * C::kBoxBytes + (ks & 3) * 32;
-          mma_bf16_ss(d_tmem, sdesc_sw128(qt + off, 16, 1024), sdesc_sw128(kslot + off, 16, 1024),
-                      idesc_s, ks > 0 ? 1u : 0u);
-        }
-        mma_commit(&s_full[t]);
-      };
-      auto issue_pv = [&](int t, int j) {
-        const uint32_t vslot = ring_addr + ((2 * j + 1) % C::kSlots) * C::kTileBytes;
-        const uint32_t p_tmem = tmem + t * 128;
-        const uint32_t o_tmem = tmem + 256 + t * 128;
-        tc_fence_after();
-        for (int ks = 0; ks < kPfN / 16; ++ks) {
-          mma_bf16_ts(o_tmem, p_tmem + ks * 8, sdesc_sw128(vslot + ks * 2048, C::kBoxBytes, 1024),
-                      idesc_o, (n_act[t] > 0 || ks > 0) ? 1u : 0u);
-        }
-      };
-
-      // Prologue: S(0) for both tiles.
-      if (ok) ok = wait_slot(0);
-      for (int t = 0; t < 2 && ok; ++t)
-        if (active(t, 0)) issue_s(t, 0);
-      for (int j = 0; j < j_count && ok; ++j) {
-        if (!(ok = wait_slot(2 * j + 1))) break;  // V_j
-        bool k_next_ready = j + 1 >= j_count;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (active(t, j)) {
-            if (!(ok = mbar_wait(&p_full[t], n_act[t] & 1, kStatusTimeoutMma))) break;
-            issue_pv(t, j);
-            ++n_act[t];
+      int ubase = 0;              // ring position of the current item's K_0
+      int nq = 0;                 // busy items started (q_full phases)
+      int n_act[2] = {0, 0};      // P tiles consumed per q tile (p_full phases)
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const PfItem it = prefill_item(p, ms, item);
+        if (!it.busy) continue;
+        if (!(ok = mbar_wait(q_full, nq & 1, kStatusTimeoutMma))) break;
+        ++nq;
+        int s_left = 0;  // S products still to issue for this item
+        for (int t = 0; t < 2; ++t)
+          for (int j = 0; j < it.j_count; ++j) s_left += tile_active(it, t, j) ? 1 : 0;
+        auto slot_addr = [&](int idx) {
+          return ring_addr + ((ubase + idx) % C::kSlots) * C::kTileBytes;
+        };
+        auto wait_slot = [&](int idx) {
+          const int u = ubase + idx;
+          return mbar_wait(&kv_full[u % C::kSlots], (u / C::kSlots) & 1, kStatusTimeoutMma);
+        };
+        auto release = [&](int idx) { mma_commit(&kv_empty[(ubase + idx) % C::kSlots]); };
+        auto issue_s = [&](int t, int j) {
+          const uint32_t kslot = slot_addr(2 * j);
+          const uint32_t qt = sq_addr + t * C::kTileBytes;
+          const uint32_t d_tmem = tmem + t * 128;
+          tc_fence_after();
+          for (int ks = 0; ks < ksteps; ++ks) {
+            const uint32_t off = (ks >> 2) * C::kBoxBytes + (ks & 3) * 32;
+            mma_bf16_ss(d_tmem, sdesc_sw128(qt + off, 16, 1024),
+                        sdesc_sw128(kslot + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
           }
-          if (j + 1 < j_count && active(t, j + 1)) {
-            if (!k_next_ready) {
-              if (!(ok = wait_slot(2 * (j + 1)))) break;  // K_{j+1}
-              k_next_ready = true;
+          mma_commit(&s_full[t]);
+          if (--s_left == 0) mma_commit(q_empty);  // Q no longer read: it may be reloaded
+        };
+        auto issue_pv = [&](int t, int j, bool first) {
+          const uint32_t vslot = slot_addr(2 * j + 1);
+          const uint32_t p_tmem = tmem + t * 128;
+          const uint32_t o_tmem = tmem + 256 + t * 128;
+          tc_fence_after();
+          for (int ks = 0; ks < kPfN / 16; ++ks)
+            mma_bf16_ts(o_tmem, p_tmem + ks * 8,
+                        sdesc_sw128(vslot + ks * 2048, C::kBoxBytes, 1024), idesc_o,
+                        (!first || ks > 0) ? 1u : 0u);
+        };
+
+        // Prologue: S(0) of the first active tile only; the other tile's S(0)
+        // follows once the first tile's P(0) is ready.
+        if (!(ok = wait_slot(0))) break;
+        const bool both0 = tile_active(it, 0, 0) && tile_active(it, 1, 0);
+        if (tile_active(it, 0, 0)) issue_s(0, 0);
+        else if (tile_active(it, 1, 0)) issue_s(1, 0);
+        bool first_pv[2] = {true, true};
+        for (int j = 0; j < it.j_count && ok; ++j) {
+          if (!(ok = wait_slot(2 * j + 1))) break;  // V_j
+          bool k_next_ready = j + 1 >= it.j_count;
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (tile_active(it, t, j)) {
+              if (!(ok = mbar_wait(&p_full[t], n_act[t] & 1, kStatusTimeoutMma))) break;
+              if (j == 0 && t == 0 && both0) issue_s(1, 0);  // delayed start of tile B
+              issue_pv(t, j, first_pv[t]);
+              first_pv[t] = false;
+              ++n_act[t];
             }
-            issue_s(t, j + 1);
+            if (j + 1 < it.j_count && tile_active(it, t, j + 1)) {
+              if (!k_next_ready) {
+                if (!(ok = wait_slot(2 * (j + 1)))) break;  // K_{j+1}
+                k_next_ready = true;
+              }
+              issue_s(t, j + 1);
+            }
           }
+          // K_{j+1} must have landed before it can be released.
+          if (ok && !k_next_ready) ok = wait_slot(2 * (j + 1));
+          if (!ok) break;
+          // Release each slot once its last reader is issued: K_0 after both
+          // S(0), V_j after P.V of iteration j, K_{j+1} after S of j+1.
+          if (j == 0) release(0);
+          release(2 * j + 1);
+          if (j + 1 < it.j_count) release(2 * (j + 1));
         }
-        // K_{j+1} must have landed before iteration j+1 can release it.
-        if (ok && !k_next_ready) ok = wait_slot(2 * (j + 1));
         if (!ok) break;
-        // Release K_j and V_j once everything issued so far has completed.
-        mma_commit(&kv_empty[(2 * j) % C::kSlots]);
-        mma_commit(&kv_empty[(2 * j + 1) % C::kSlots]);
+        mma_commit(&o_done[0]);
+        mma_commit(&o_done[1]);
+        ubase += 2 * it.j_count;
       }
-      mma_commit(&o_done[0]);
-      mma_commit(&o_done[1]);
       // Drain: every MMA finished before TMEM can be released.
       mma_commit(drain);
       mbar_wait(drain, 0, kStatusTimeoutMma);
@@ -297,138 +350,231 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     // ------------------------------------------------------------ softmax / epilogue
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
     const int t = (warp - 4) / 4;            // tile 0 (A) or 1 (B)
-    const TileInfo& ti = t == 0 ? ta : tb;
     const int quarter = warp & 3;            // TMEM lane quarter of this warp
     const int r = quarter * 32 + lane;       // row within the tile
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t s_tmem = tmem + lane_base + t * 128;
     const uint32_t o_tmem = tmem + lane_base + 256 + t * 128;
-    const long long grow = (long long)ti.row0 + r;  // row within the unit
-    const bool row_valid = r < ti.nrows;
-    int lo = 0, hi = -1;
-    if (row_valid) {
-      const int qpos = p.kv_len - p.q_len + (int)(grow % p.q_len);
-      lo = first_key(ms, qpos);
-      hi = last_key(ms, qpos);
-    }
-    float m_run = -INFINITY, l_run = 0.f;
-    int n_act = 0;
+    int n_act = 0;   // S tiles consumed (s_full phases)
+    int n_done = 0;  // busy items finished (o_done phases)
     bool ok = true;
-    for (int j = 0; j < j_count && ok; ++j) {
-      const int jj = j_first + j;
-      if (ti.kr.t_count == 0 || jj < ti.kr.t_first || jj >= ti.kr.t_first + ti.kr.t_count)
-        continue;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], n_act & 1, kStatusTimeoutSoftmax));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t s0[32], s1[32], s2[32], s3[32];
-      tmem_ld32(s_tmem + 0, s0);
-      tmem_ld32(s_tmem + 32, s1);
-      tmem_ld32(s_tmem + 64, s2);
-      tmem_ld32(s_tmem + 96, s3);
-      tmem_ld_wait();
-      float x[128];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        x[c] = __uint_as_float(s0[c]);
-        x[32 + c] = __uint_as_float(s1[c]);
-        x[64 + c] = __uint_as_float(s2[c]);
-        x[96 + c] = __uint_as_float(s3[c]);
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const PfItem it = prefill_item(p, ms, item);
+      const TileInfo ti = t == 0 ? it.tile[0] : it.tile[1];
+      const long long grow = (long long)ti.row0 + r;  // row within the unit
+      const bool row_valid = r < ti.nrows;
+      int lo = 0, hi = -1;
+      if (row_valid) {
+        const int qpos = p.kv_len - p.q_len + (int)(grow % p.q_len);
+        lo = first_key(ms, qpos);
+        hi = last_key(ms, qpos);
       }
-      const int key0 = jj * kPfN;
-      const bool need_mask = !(key0 >= ti.kr.all_lo && key0 + kPfN - 1 <= ti.kr.all_hi);
-      if (p.use_softcap) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = p.cap_out * tanh_accurate(x[c] * p.cap_in);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] *= p.logit_scale;
-      }
-      if (need_mask) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (key0 + c < lo || key0 + c > hi) x[c] = -INFINITY;
-      }
-      float mt = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) mt = fmaxf(mt, x[c]);
-      // Rescale only when the max grew by more than 2^8 (or was -inf): the
-      // stale max keeps p <= 256, and O / l stays consistent either way.
-      const float m_new = fmaxf(m_run, mt);
-      const bool need =
-          (m_new > m_run + kRescaleThreshold) || (m_run == -INFINITY && m_new != -INFINITY);
-      const float alpha = need ? ex2(m_run - m_new) : 1.0f;  // 0 when m_run = -inf
-      if (need) {
-        l_run *= alpha;
-        m_run = m_new;
-      }
-      if (__any_sync(0xffffffffu, need) && n_act > 0) {
-        // tcgen05.ld/st are warp-collective: every lane takes part.
-        for (int c0 = 0; c0 < p.d_pad; c0 += 16) {
-          uint32_t ov[16];
-          tmem_ld16(o_tmem + c0, ov);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st16(o_tmem + c0, ov);
-        }
-        tmem_st_wait();
-      }
-      const float base = m_run == -INFINITY ? 0.f : m_run;
-      float ls = 0.f;
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const float p0 = ex2(x[32 * q4 + 2 * c] - base);
-          const float p1 = ex2(x[32 * q4 + 2 * c + 1] - base);
-          ls += p0 + p1;
-          pk[c] = pack_bf16(p0, p1);
-        }
-        tmem_st16(s_tmem + 16 * q4, pk);
-      }
-      l_run += ls;
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
-      ++n_act;
-    }
-    // ---- epilogue: o = O / l, bf16, one row per thread (warp-collective loads)
-    if (__all_sync(0xffffffffu, ok) && ti.nrows > 0) {
-      const bool have = n_act > 0;
-      bool ready = true;
-      if (have) {
-        ready = __all_sync(0xffffffffu, mbar_wait(&o_done[t], 0, kStatusTimeoutEpilogue));
+      float m_run = -INFINITY, l_run = 0.f;
+      int act = 0;  // key tiles this q tile consumed in this item
+      for (int j = 0; j < it.j_count && ok; ++j) {
+        if (!tile_active(it, t, j)) continue;
+        const int jj = it.j_first + j;
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], n_act & 1, kStatusTimeoutSoftmax));
+        if (!ok) break;
         tc_fence_after();
-      }
-      if (ready) {
-        const bool live = have && l_run > 0.f;
-        const float inv = live ? 1.0f / l_run : 0.f;
-        __nv_bfloat16* orow = p.o + ((long long)unit * p.rows + grow) * p.head_dim;
-        for (int c0 = 0; c0 < p.head_dim; c0 += 16) {
-          uint32_t ov[16];
+        uint32_t s0[32], s1[32], s2[32], s3[32];
+        tmem_ld32(s_tmem + 0, s0);
+        tmem_ld32(s_tmem + 32, s1);
+        tmem_ld32(s_tmem + 64, s2);
+        tmem_ld32(s_tmem + 96, s3);
+        tmem_ld_wait();
+        float x[128];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) ov[e] = 0u;
-          if (have) {
+        for (int c = 0; c < 32; ++c) {
+          x[c] = __uint_as_float(s0[c]);
+          x[32 + c] = __uint_as_float(s1[c]);
+          x[64 + c] = __uint_as_float(s2[c]);
+          x[96 + c] = __uint_as_float(s3[c]);
+        }
+        const int key0 = jj * kPfN;
+        const bool need_mask = !(key0 >= ti.kr.all_lo && key0 + kPfN - 1 <= ti.kr.all_hi);
+        // Softcap: when every |score| of the warp's rows maps to |y| <= 1/2 the
+        // tanh runs as a polynomial on the FMA pipe, leaving MUFU to ex2.
+        bool small_y = false;
+        if constexpr (kCap) {
+          float am[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) am[i] = fabsf(x[i]);
+#pragma unroll
+          for (int c = 8; c < 128; ++c) am[c & 7] = fmaxf(am[c & 7], fabsf(x[c]));
+          const float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])),
+                                   fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
+          small_y = __all_sync(0xffffffffu, amax * p.cap_in <= 0.5f);
+        }
+        if (need_mask) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (key0 + c < lo || key0 + c > hi) x[c] = -INFINITY;
+        }
+        // Row max of the raw scores (a tree of 8 chains); scale and softcap
+        // are increasing, so the log2-domain max is the transform of this one.
+        float mx[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = x[i];
+#pragma unroll
+        for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+        const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        const float mt = mraw == -INFINITY ? -INFINITY
+                         : kCap ? p.cap_out * (small_y ? tanh_poly_small(mraw * p.cap_in)
+                                                       : tanh_fast(mraw * p.cap_in))
+                                : mraw * p.logit_scale;
+        // Rescale only when the max grew by more than 2^8 (or was -inf): the
+        // stale max keeps p <= 256, and O / l stays consistent either way.
+        const float m_new = fmaxf(m_run, mt);
+        const bool need =
+            (m_new > m_run + kRescaleThreshold) || (m_run == -INFINITY && m_new != -INFINITY);
+        const float alpha = need ? ex2(m_run - m_new) : 1.0f;  // 0 when m_run = -inf
+        if (need) {
+          l_run *= alpha;
+          m_run = m_new;
+        }
+        if (__any_sync(0xffffffffu, need) && act > 0) {
+          // tcgen05.ld/st are warp-collective: every lane takes part.
+          for (int c0 = 0; c0 < p.d_pad; c0 += 16) {
+            uint32_t ov[16];
             tmem_ld16(o_tmem + c0, ov);
             tmem_ld_wait();
-          }
-          uint32_t w[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float a = live ? __uint_as_float(ov[2 * e]) * inv : 0.f;
-            const float b = live ? __uint_as_float(ov[2 * e + 1]) * inv : 0.f;
-            w[e] = pack_bf16(a, b);
+            for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st16(o_tmem + c0, ov);
           }
-          if (row_valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c0);
-            dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            if (c0 + 16 <= p.head_dim) dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          tmem_st_wait();
+        }
+        const float base = m_run == -INFINITY ? 0.f : m_run;
+        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // p = 2^(logit - base) as bf16 pairs into TMEM over S (P chunk q of 32
+        // keys lands in columns [16q, 16q + 16), whose scores are consumed).
+        if (!kCap || small_y) {
+          // Common case: fully unrolled over the scores already in registers;
+          // on mask tiles the logit of a hidden key is forced to -inf.
+          const int clo = lo - key0, chi = hi - key0;  // visible columns
+          auto emit = [&](auto masked) {
+#pragma unroll
+            for (int q4 = 0; q4 < 4; ++q4) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                float pe[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const int col = 32 * q4 + 2 * c + h;
+                  float a;
+                  if constexpr (kCap)
+                    a = fmaf(p.cap_out, tanh_poly_small(x[col] * p.cap_in), -base);
+                  else
+                    a = fmaf(x[col], p.logit_scale, -base);
+                  if (masked(col)) a = -INFINITY;
+                  pe[h] = ex2(a);
+                }
+                ls[c & 7] += pe[0] + pe[1];
+                pk[c] = pack_bf16(pe[0], pe[1]);
+              }
+              tmem_st16(s_tmem + 16 * q4, pk);
+            }
+          };
+          if (need_mask)
+            emit([&](int col) { return col < clo || col > chi; });
+          else
+            emit([](int) { return false; });
+        } else {
+          // Softcap with large arguments (hardware tanh): a compact loop over
+          // 32 scores at a time re-read from TMEM; hidden keys get p = 0.
+          const int clo = need_mask ? lo - key0 : 0;
+          const int chi = need_mask ? hi - key0 : kPfN - 1;
+#pragma unroll 1
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t sv[32];
+            tmem_ld32(s_tmem + 32 * q4, sv);
+            tmem_ld_wait();
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              float pe[2];
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int col = 32 * q4 + 2 * c + h;
+                const float a =
+                    fmaf(p.cap_out, tanh_fast(__uint_as_float(sv[2 * c + h]) * p.cap_in), -base);
+                pe[h] = (col < clo || col > chi) ? 0.f : ex2(a);
+              }
+              ls[c & 7] += pe[0] + pe[1];
+              pk[c] = pack_bf16(pe[0], pe[1]);
+            }
+            tmem_st16(s_tmem + 16 * q4, pk);
+          }
+        }
+        l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+        ++n_act;
+        ++act;
+      }
+      if (!ok) break;
+      // ---- epilogue: o = O / l as bf16, one row per thread.  The next item's
+      // first P.V may overwrite O only after this warpgroup's next P arrival,
+      // which follows these (waited) TMEM loads in program order.
+      if (it.busy) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], n_done & 1, kStatusTimeoutEpilogue));
+        ++n_done;
+        if (!ok) break;
+        tc_fence_after();
+      }
+      if (ti.nrows > 0) {
+        // o = O / l as bf16 into this warp's 128B-swizzled 32-row staging box,
+        // 64 columns at a time, each written out by one TMA store (rows past
+        // the unit's end are not written).
+        const bool have = act > 0;
+        const bool live = have && l_run > 0.f;
+        const float inv = live ? 1.0f / l_run : 0.f;
+        uint8_t* stage = stage_all + (t * 4 + quarter) * 4096;
+        for (int c0 = 0; c0 < p.d_pad; c0 += 64) {
+          const int ncols = min(64, p.d_pad - c0);
+          if (lane == 0) bulk_wait_read();  // previous store has read the box
+          __syncwarp();
+          for (int c1 = 0; c1 < ncols; c1 += 32) {
+            uint32_t ov[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = 0u;
+            if (have) {
+              if (ncols - c1 >= 32) {
+                tmem_ld32(o_tmem + c0 + c1, ov);
+              } else {
+                tmem_ld16(o_tmem + c0 + c1, *reinterpret_cast<uint32_t(*)[16]>(ov));
+              }
+              tmem_ld_wait();
+            }
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {  // 8 columns = one 16-byte chunk
+              if (c1 + 8 * g < ncols) {
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float a = live ? __uint_as_float(ov[8 * g + 2 * e]) * inv : 0.f;
+                  const float b = live ? __uint_as_float(ov[8 * g + 2 * e + 1]) * inv : 0.f;
+                  w[e] = pack_bf16(a, b);
+                }
+                *reinterpret_cast<uint4*>(stage + sw128(lane, (c1 >> 3) + g)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tm_o, stage, c0, ti.row0 + quarter * 32, it.unit);
+            bulk_commit();
           }
         }
       }
     }
+    if (lane == 0) bulk_wait_all();  // stores done before the CTA exits
   }
 
   // ---------------------------------------------------------------- teardown

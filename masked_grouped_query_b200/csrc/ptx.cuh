@@ -69,6 +69,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
 }
 
 // ---------------------------------------------------------------- TMA
+// Byte offset of (row, 16-byte chunk) inside a 64-column bf16 tile written by
+// TMA with 128-byte swizzle (1024-byte aligned): chunk index XOR (row % 8).
+__device__ __forceinline__ uint32_t sw128(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(map) : "memory");
 }
@@ -82,6 +88,32 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
       "l"(map), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
       : "memory");
+}
+
+// 3-D tiled bulk tensor store shared -> global, bulk-group completion.
+// Elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y,
+                                             int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(map),
+      "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until this thread's committed bulk stores have read their shared memory.
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until this thread's committed bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Order this thread's generic-proxy shared-memory writes before later
+// async-proxy (TMA) reads of them.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05
@@ -250,6 +282,16 @@ __device__ __forceinline__ float tanh_accurate(float y) {
   const float t = 1.0f - 2.0f * rcp(e + 1.0f);
   return copysignf(t, y);
 }
+// tanh(y) for |y| <= 1/2 on the FMA pipe: y * P(y^2) with a cubic P fitted
+// for least maximum absolute error on [0, 1/2] (1.7e-7; fit_tanh_poly.py
+// next to this file).  Outside that range use tanh_fast / tanh_accurate.
+__device__ __forceinline__ float tanh_poly_small(float y) {
+  const float y2 = y * y;
+  return y * fmaf(fmaf(fmaf(-0.04341723769903183f, y2, 0.13148456811904907f), y2,
+                       -0.3332125246524811f),
+                  y2, 0.9999978542327881f);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);

@@ -61,13 +61,18 @@ def test_static_scratch_matches_gqa_attn_fwd_twice(w):
 
 def test_static_scratch_rejects_plans_beyond_its_size():
     lib = _lib.load()
-    # 32 (batch, kv head) units x 17 splits x 64 rows of fp32 partials (~18 MB) > 8 MiB.
-    w = Workload("big", 8, 4, 8192, 64, 4, 128, True, 4096, 30.0, 44)
+    # One key tile per split (the tuning override) at head_dim 256 and 64 rows
+    # per kv head: 2 kv heads x 128 splits x 64 rows x 256 fp32 = 16.8 MB > 8 MiB.
+    w = Workload("big", 1, 4, 8192, 32, 2, 256, True, None, None, 44)
     q = torch.zeros(w.batch, w.num_q_heads, w.q_len, w.head_dim, dtype=torch.bfloat16,
                     device="cuda")
     k = torch.zeros(w.batch, w.num_kv_heads, w.kv_len, w.head_dim, dtype=torch.bfloat16,
                     device="cuda")
     out = torch.empty_like(q)
-    rc = _call(lib.gqa_attn_fwd_static_scratch, w, q, k, k, out)
+    assert lib.gqa_attn_set_override(2, 1) == 0
+    try:
+        rc = _call(lib.gqa_attn_fwd_static_scratch, w, q, k, k, out)
+    finally:
+        lib.gqa_attn_set_override(2, 0)
     assert rc == -10
     assert "static scratch too small" in lib.gqa_attn_last_error_detail().decode()
