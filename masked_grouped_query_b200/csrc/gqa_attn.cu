@@ -188,7 +188,7 @@ int plan_decode(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
   return GQA_ATTN_OK;
 }
 
-int plan_prefill(const Problem& pr, Plan* pl) {
+int plan_prefill(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
   pl->path = kPathPrefill;
   pl->dch = pr.d <= 64 ? 1 : 2;
   pl->d_pad = (pr.d + 15) / 16 * 16;
@@ -206,7 +206,24 @@ int plan_prefill(const Problem& pr, Plan* pl) {
     if (kr.t_count > max_tiles) max_tiles = kr.t_count;
   }
   pl->max_tiles = max_tiles;
+  // Too few tile pairs to fill the GPU (multi-token decode shapes): split each
+  // pair's key range so that about one item per SM runs; the splits' partials
+  // are merged by the last split to finish.
+  const long long pairs = pl->ctas;
+  pl->splits = 1;
+  if (pairs < dev.sms && max_tiles > 1) {
+    long long s = dev.sms / (pairs > 0 ? pairs : 1);
+    if (s > max_tiles) s = max_tiles;
+    pl->splits = (int)(s < 1 ? 1 : s);
+  }
+  pl->ctas = pairs * pl->splits;
   if (pl->ctas > 0x7fffffffLL) return GQA_ATTN_ERR_TOO_LARGE;
+  if (pl->splits > 1) {
+    pl->ws_bytes = align256((size_t)pairs * 2 * pl->splits * (size_t)pl->d_pad * kPfM * 4);
+    pl->off_lse = pl->ws_bytes;
+    pl->ws_bytes += align256((size_t)pairs * 2 * pl->splits * 2 * kPfM * 4);
+    pl->ticket_bytes = align256((size_t)pairs * 2 * 4 * sizeof(unsigned int));
+  }
   return GQA_ATTN_OK;
 }
 
@@ -219,15 +236,16 @@ int make_plan(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
     pl->path = kPathZero;
     return GQA_ATTN_OK;
   }
-  // Short query blocks (<= 64 rows per kv head) are K/V-bandwidth bound: the
-  // split-KV decode kernel.  Longer ones go to the tcgen05 kernel (head_dim
-  // up to 128); the decode kernel also covers head_dim 136..256.
+  // Up to 16 rows per kv head (single-token decode) run on the split-KV
+  // mma.sync decode kernel; more rows on the tcgen05 kernel (head_dim up to
+  // 128), with key-range splits when there are few row tiles; the decode
+  // kernel also covers head_dim 136..256.
   const int forced = g_force_path.load();
   const bool prefill_ok = pr.d <= 128;
-  bool prefill = pr.rows > kDecRows && prefill_ok;
+  bool prefill = pr.rows > 16 && prefill_ok;
   if (forced == 1) prefill = false;
   if (forced == 2 && prefill_ok) prefill = true;
-  return prefill ? plan_prefill(pr, pl) : plan_decode(pr, dev, pl);
+  return prefill ? plan_prefill(pr, dev, pl) : plan_decode(pr, dev, pl);
 }
 
 // ------------------------------------------------------------------ workspace
@@ -375,7 +393,8 @@ int launch_decode(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void
 
 template <int DCH, bool kCap>
 int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
-                     const void* k, const void* v, void* o, cudaStream_t stream) {
+                     const void* k, const void* v, void* o, void* ws, void* tickets,
+                     cudaStream_t stream) {
   using C = PrefillCfg<DCH>;
   if (!dev.prefill_attr[(DCH - 1) + (kCap ? 2 : 0)]) {
     // The register split inside the kernel must fit what the block is
@@ -408,7 +427,11 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.rows = (int)pr.rows;
   p.tiles_per_unit = pl.tiles_per_unit;
   p.pairs_per_unit = pl.pairs_per_unit;
+  p.splits = pl.splits;
   p.n_items = (int)pl.ctas;
+  p.ws_o = (float*)ws;
+  p.ws_ml = ws ? (float*)((char*)ws + pl.off_lse) : nullptr;
+  p.tickets = (unsigned int*)tickets;
   p.pair_heads = pl.pair_heads;
   p.causal = pr.causal;
   p.window = pr.window;
@@ -425,12 +448,13 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
 }
 
 int launch_prefill(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
-                   const void* k, const void* v, void* o, cudaStream_t stream) {
+                   const void* k, const void* v, void* o, void* ws, void* tickets,
+                   cudaStream_t stream) {
   if (pr.softcap > 0.f)
-    return pl.dch == 1 ? launch_prefill_d<1, true>(pr, pl, dev, q, k, v, o, stream)
-                       : launch_prefill_d<2, true>(pr, pl, dev, q, k, v, o, stream);
-  return pl.dch == 1 ? launch_prefill_d<1, false>(pr, pl, dev, q, k, v, o, stream)
-                     : launch_prefill_d<2, false>(pr, pl, dev, q, k, v, o, stream);
+    return pl.dch == 1 ? launch_prefill_d<1, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
+                       : launch_prefill_d<2, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+  return pl.dch == 1 ? launch_prefill_d<1, false>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
+                     : launch_prefill_d<2, false>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
 }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -469,8 +493,6 @@ int run(const Problem& pr, const void* q, const void* k, const void* v, void* o,
       return cudaMemsetAsync(o, 0, bytes, stream) == cudaSuccess ? GQA_ATTN_OK
                                                                  : GQA_ATTN_ERR_LAUNCH;
     }
-    case kPathPrefill:
-      return launch_prefill(pr, pl, *dev, q, k, v, o, stream);
     default: {
       void* ws = nullptr;
       void* tickets = nullptr;
@@ -478,6 +500,7 @@ int run(const Problem& pr, const void* q, const void* k, const void* v, void* o,
         rc = get_workspace(stream, pl.ws_bytes, pl.ticket_bytes, &ws, &tickets);
         if (rc != GQA_ATTN_OK) return rc;
       }
+      if (pl.path == kPathPrefill) return launch_prefill(pr, pl, *dev, q, k, v, o, ws, tickets, stream);
       return launch_decode(pr, pl, *dev, q, k, v, o, ws, tickets, stream);
     }
   }

@@ -60,11 +60,18 @@ struct PrefillParams {
   int q_len, kv_len, head_dim, d_pad;
   int rows;              // rows per unit: group * q_len
   int tiles_per_unit;    // ceil(rows / 128)
-  int pairs_per_unit;    // work items per unit
-  int n_items;           // units * pairs_per_unit
+  int pairs_per_unit;    // tile pairs per unit
+  int splits;            // key-range splits per tile pair (1 = none)
+  int n_items;           // units * pairs_per_unit * splits
   int pair_heads;        // 1: tiles (2p, 2p+1) are two heads at one position
   int causal, window;
   float logit_scale, cap_in, cap_out;
+  // Split partials (splits > 1): per (pair, tile, split) O as fp32 [d][128
+  // rows] (column-major, so a warp's accesses coalesce) and (m, l) per row;
+  // tickets per (pair, tile, warp) count the splits that have finished.
+  float* ws_o;
+  float* ws_ml;
+  unsigned int* tickets;
 };
 
 template <int DCH>
@@ -112,11 +119,13 @@ __device__ __forceinline__ TileInfo prefill_tile(const PrefillParams& p, const M
   return ti;
 }
 
-// One work item: a unit and its pair of q tiles, with the union of their
-// key-tile ranges [j_first, j_first + j_count).  An item without key tiles
-// is not "busy": its rows (if any) are written as zeros without MMAs.
+// One work item: a unit, its pair of q tiles and one split of the union of
+// their key-tile ranges: key tiles [j_first, j_first + j_count).  An item
+// without key tiles is not "busy": no loads or MMAs run for it.
 struct PfItem {
   int unit;
+  int pair_index;  // unit * pairs_per_unit + pair
+  int split;
   TileInfo tile[2];
   int j_first, j_count;
   bool busy;
@@ -125,8 +134,10 @@ struct PfItem {
 __device__ __forceinline__ PfItem prefill_item(const PrefillParams& p, const MaskSpec& ms,
                                                int item) {
   PfItem it;
-  it.unit = item / p.pairs_per_unit;
-  const int pair = item % p.pairs_per_unit;
+  it.split = item % p.splits;
+  it.pair_index = item / p.splits;
+  it.unit = it.pair_index / p.pairs_per_unit;
+  const int pair = it.pair_index % p.pairs_per_unit;
   it.tile[0] = prefill_tile(p, ms, pair, 0);
   it.tile[1] = prefill_tile(p, ms, pair, 1);
   const KeyRange& a = it.tile[0].kr;
@@ -140,6 +151,12 @@ __device__ __forceinline__ PfItem prefill_item(const PrefillParams& p, const Mas
     const int lb = b.t_count ? b.t_first + b.t_count - 1 : -1;
     it.j_first = min(fa, fb);
     it.j_count = max(la, lb) - it.j_first + 1;
+  }
+  if (p.splits > 1) {  // this item's share of the key tiles
+    const int per = (it.j_count + p.splits - 1) / p.splits;
+    const int js = min(it.j_count, it.split * per), je = min(it.j_count, js + per);
+    it.j_first += js;
+    it.j_count = je - js;
   }
   it.busy = it.j_count > 0;
   return it;
@@ -527,49 +544,103 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         tc_fence_after();
       }
       if (ti.nrows > 0) {
-        // o = O / l as bf16 into this warp's 128B-swizzled 32-row staging box,
-        // 64 columns at a time, each written out by one TMA store (rows past
-        // the unit's end are not written).
         const bool have = act > 0;
-        const bool live = have && l_run > 0.f;
-        const float inv = live ? 1.0f / l_run : 0.f;
         uint8_t* stage = stage_all + (t * 4 + quarter) * 4096;
-        for (int c0 = 0; c0 < p.d_pad; c0 += 64) {
-          const int ncols = min(64, p.d_pad - c0);
-          if (lane == 0) bulk_wait_read();  // previous store has read the box
-          __syncwarp();
-          for (int c1 = 0; c1 < ncols; c1 += 32) {
-            uint32_t ov[32];
+        // Write this warp's 32 output rows as bf16: through its 128B-swizzled
+        // 32-row staging box, 64 columns at a time, each written out by one
+        // TMA store (rows past the unit's end are not written).  value16(col,
+        // v) fills v with the fp32 outputs of columns col .. col + 15.
+        auto store_rows = [&](auto value16) {
+          for (int c0 = 0; c0 < p.d_pad; c0 += 64) {
+            const int ncols = min(64, p.d_pad - c0);
+            if (lane == 0) bulk_wait_read();  // the previous store has read the box
+            __syncwarp();
+            for (int c1 = 0; c1 < ncols; c1 += 16) {
+              float v[16];
+              value16(c0 + c1, v);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = 0u;
-            if (have) {
-              if (ncols - c1 >= 32) {
-                tmem_ld32(o_tmem + c0 + c1, ov);
-              } else {
-                tmem_ld16(o_tmem + c0 + c1, *reinterpret_cast<uint32_t(*)[16]>(ov));
+              for (int g = 0; g < 2; ++g) {  // 8 columns = one 16-byte chunk
+                const uint4 w = make_uint4(pack_bf16(v[8 * g], v[8 * g + 1]),
+                                           pack_bf16(v[8 * g + 2], v[8 * g + 3]),
+                                           pack_bf16(v[8 * g + 4], v[8 * g + 5]),
+                                           pack_bf16(v[8 * g + 6], v[8 * g + 7]));
+                *reinterpret_cast<uint4*>(stage + sw128(lane, (c1 >> 3) + g)) = w;
               }
-              tmem_ld_wait();
             }
-#pragma unroll
-            for (int g = 0; g < 4; ++g) {  // 8 columns = one 16-byte chunk
-              if (c1 + 8 * g < ncols) {
-                uint32_t w[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float a = live ? __uint_as_float(ov[8 * g + 2 * e]) * inv : 0.f;
-                  const float b = live ? __uint_as_float(ov[8 * g + 2 * e + 1]) * inv : 0.f;
-                  w[e] = pack_bf16(a, b);
-                }
-                *reinterpret_cast<uint4*>(stage + sw128(lane, (c1 >> 3) + g)) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
-              }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tm_o, stage, c0, ti.row0 + quarter * 32, it.unit);
+              bulk_commit();
             }
           }
-          fence_proxy_async_smem();
+        };
+        // O columns col .. col + 15 of this thread's row from TMEM (warp-collective).
+        auto load_o = [&](int col, float (&v)[16]) {
+          uint32_t ov[16];
+          tmem_ld16(o_tmem + col, ov);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(ov[e]);
+        };
+        if (p.splits == 1) {
+          const bool live = have && l_run > 0.f;
+          const float inv = live ? 1.0f / l_run : 0.f;
+          store_rows([&](int col, float (&v)[16]) {
+            if (have) {
+              load_o(col, v);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = live ? v[e] * inv : 0.f;
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            }
+          });
+        } else {
+          // Split partial: O (unnormalised), m, l of this split; the warp
+          // that finishes a row group's last split merges all of them.
+          const long long blk = (long long)(it.pair_index * 2 + t) * p.splits;
+          float* po = p.ws_o + (blk + it.split) * (long long)p.d_pad * kPfM;
+          float* pml = p.ws_ml + (blk + it.split) * 2 * kPfM;
+          for (int c0 = 0; c0 < p.d_pad && have; c0 += 16) {
+            float v[16];
+            load_o(c0, v);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) po[(long long)(c0 + e) * kPfM + r] = v[e];
+          }
+          pml[r] = have ? m_run : -INFINITY;
+          pml[kPfM + r] = have ? l_run : 0.f;
+          __threadfence();
           __syncwarp();
-          if (lane == 0) {
-            tma_store_3d(&tm_o, stage, c0, ti.row0 + quarter * 32, it.unit);
-            bulk_commit();
+          unsigned int ticket = 0;
+          unsigned int* tk = p.tickets + (it.pair_index * 2 + t) * 4 + quarter;
+          if (lane == 0) ticket = atomicAdd(tk, 1u);
+          ticket = __shfl_sync(0xffffffffu, ticket, 0);
+          if (ticket == (unsigned)p.splits - 1) {
+            __threadfence();
+            float M = -INFINITY;
+            for (int sp = 0; sp < p.splits; ++sp)
+              M = fmaxf(M, __ldcg(p.ws_ml + (blk + sp) * 2 * kPfM + r));
+            float L = 0.f;
+            for (int sp = 0; sp < p.splits; ++sp) {
+              const float* ml = p.ws_ml + (blk + sp) * 2 * kPfM;
+              const float m = __ldcg(ml + r);
+              L += m == -INFINITY ? 0.f : ex2(m - M) * __ldcg(ml + kPfM + r);
+            }
+            const float inv = L > 0.f ? 1.0f / L : 0.f;
+            store_rows([&](int col, float (&v)[16]) {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = 0.f;
+              for (int sp = 0; sp < p.splits; ++sp) {
+                const float m = __ldcg(p.ws_ml + (blk + sp) * 2 * kPfM + r);
+                if (m == -INFINITY) continue;  // empty split: its O was never written
+                const float w = ex2(m - M) * inv;
+                const float* src = p.ws_o + (blk + sp) * (long long)p.d_pad * kPfM + r;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] += w * __ldcg(src + (long long)(col + e) * kPfM);
+              }
+            });
+            if (lane == 0) atomicExch(tk, 0u);  // ready for the next call
           }
         }
       }

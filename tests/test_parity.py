@@ -174,12 +174,37 @@ def test_deterministic(name):
 
 @pytest.mark.parametrize("tps", [1, 3, 7, 1000])
 def test_forced_split_geometries_agree_with_oracle(tps):
+    # The split-KV decode kernel, forced, at several split sizes.
     w = WORKLOADS["long_context_decode_16to1"].with_(batch=2)
+    mgq.set_override("force_path", 1)
     mgq.set_override("tiles_per_split", tps)
     try:
         check_workload(w)
     finally:
         mgq.set_override("tiles_per_split", 0)
+        mgq.set_override("force_path", 0)
+
+
+@pytest.mark.parametrize("cfg", [
+    (8, 4, 32768, 64, 4, 128, True, 4096, 30.0),   # the 16:1 long-context decode shape
+    (2, 20, 3000, 8, 2, 128, True, None, None),     # 80 rows per kv head
+    (1, 3, 1000, 16, 1, 72, False, 300, None),      # window without causal, D = 72
+    (3, 2, 777, 32, 2, 64, True, None, 20.0),       # ragged keys, D = 64
+])
+def test_tcgen05_key_splits(cfg):
+    # Few row tiles: the tcgen05 kernel splits each tile pair's key range
+    # and merges the partials; the plan must actually split.
+    b, lq, lk, hq, hkv, d, causal, window, cap = cfg
+    w = Workload("ks", b, lq, lk, hq, hkv, d, causal, window, cap, seed=lk + d)
+    plan = mgq.describe(b, lq, lk, hq, hkv, d, causal, window, cap)
+    assert plan["path"] == "prefill" and plan["splits"] > 1, plan
+    check_workload(w)
+    q, k, v = make_inputs(w)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    a = mgq.attention(q, k, v, causal=causal, window=window, softcap=cap)
+    b2 = mgq.attention(q, k, v, causal=causal, window=window, softcap=cap)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b2)  # deterministic merge order
 
 
 def test_host_buffer_entry_point_matches_device_entry_point():
