@@ -133,9 +133,10 @@ def describe(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, causal=F
 
 
 def set_override(key: str, value: int) -> None:
-    """Test/tuning knob: ``force_path`` (0 auto, 1 decode, 2 prefill) or
-    ``tiles_per_split`` (0 = automatic)."""
-    k = {"force_path": 1, "tiles_per_split": 2}[key]
+    """Test/tuning knob: ``force_path`` (0 auto, 1 decode, 2 prefill),
+    ``tiles_per_split`` (decode, 0 = automatic) or ``prefill_splits``
+    (tcgen05 kernel, units with one row tile; 0 = automatic)."""
+    k = {"force_path": 1, "tiles_per_split": 2, "prefill_splits": 3}[key]
     _lib.check(_lib.load().gqa_attn_set_override(k, int(value)), "gqa_attn_set_override")
 
 

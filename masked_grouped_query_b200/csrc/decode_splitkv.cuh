@@ -189,9 +189,16 @@ __global__ void __maxnreg__(kT ? 128 : 255)
       }
       // ---- logits: element e is (key g + 8*(e>>1), row 2*t4 + (e&1))
       float x[4];
+      bool small = true;
+      if (p.use_softcap) {
+        const float am = fmaxf(fmaxf(fabsf(sc[0]), fabsf(sc[1])), fmaxf(fabsf(sc[2]), fabsf(sc[3])));
+        small = __all_sync(0xffffffffu, am * p.cap_in <= 0.5f);
+      }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        float v = p.use_softcap ? p.cap_out * tanh_accurate(sc[e] * p.cap_in) : sc[e] * p.logit_scale;
+        float v = !p.use_softcap ? sc[e] * p.logit_scale
+                  : small        ? p.cap_out * tanh_poly_small(sc[e] * p.cap_in)
+                                 : p.cap_out * tanh_fast(sc[e] * p.cap_in);
         if (need_mask) {
           const int j = key0 + wkey0 + g + 8 * (e >> 1);
           if (j < lo[e & 1] || j > hi[e & 1]) v = -INFINITY;
@@ -330,43 +337,62 @@ __global__ void __maxnreg__(kT ? 128 : 255)
           mma_16816(sc[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b2, b3);
         }
       }
-      // ---- logits (log2 domain), softcap, mask
+      // ---- logits (log2 domain), softcap, mask.  With a softcap the tanh is
+      // an FMA-pipe polynomial when every |x / s| of the warp is <= 1/2.
       float x[2][4];
+      if (p.use_softcap) {
+        float am = 0.f;
 #pragma unroll
-      for (int n = 0; n < 2; ++n)
+        for (int n = 0; n < 2; ++n)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          float v = sc[n][e];
-          v = p.use_softcap ? p.cap_out * tanh_accurate(v * p.cap_in) : v * p.logit_scale;
-          if (need_mask) {
+          for (int e = 0; e < 4; ++e) am = fmaxf(am, fabsf(sc[n][e]));
+        if (__all_sync(0xffffffffu, am * p.cap_in <= 0.5f)) {
+#pragma unroll
+          for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[n][e] = p.cap_out * tanh_poly_small(sc[n][e] * p.cap_in);
+        } else {
+#pragma unroll
+          for (int n = 0; n < 2; ++n)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) x[n][e] = p.cap_out * tanh_fast(sc[n][e] * p.cap_in);
+        }
+      } else {
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) x[n][e] = sc[n][e] * p.logit_scale;
+      }
+      if (need_mask) {
+#pragma unroll
+        for (int n = 0; n < 2; ++n)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
             const int j = key0 + wkey0 + kk * 16 + n * 8 + 2 * (lane & 3) + (e & 1);
             const int h = e >> 1;
-            if (j < lo[h] || j > hi[h]) v = -INFINITY;
+            if (j < lo[h] || j > hi[h]) x[n][e] = -INFINITY;
           }
-          x[n][e] = v;
-        }
-      // ---- online softmax update (two rows per thread, quad-wide max)
-      float mt[2];
+      }
+      // ---- online softmax update (two rows per thread, quad-wide max);
+      // O is rescaled only when a row max grows by more than 2^8.
+      float base[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         float m = fmaxf(fmaxf(x[0][2 * h], x[0][2 * h + 1]), fmaxf(x[1][2 * h], x[1][2 * h + 1]));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-        mt[h] = m;
-      }
-      float base[2];
+        const float m_new = fmaxf(m_run[h], m);
+        if (m_new > m_run[h] + 8.0f || (m_run[h] == -INFINITY && m_new != -INFINITY)) {
+          const float alpha = ex2(m_run[h] - m_new);  // 0 when m_run = -inf
+          m_run[h] = m_new;
+          l_run[h] *= alpha;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const float m_new = fmaxf(m_run[h], mt[h]);
-        base[h] = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = ex2(m_run[h] - base[h]);
-        m_run[h] = m_new;
-        l_run[h] *= alpha;
-#pragma unroll
-        for (int n = 0; n < 2 * KS; ++n) {
-          o_acc[n][2 * h] *= alpha;
-          o_acc[n][2 * h + 1] *= alpha;
+          for (int n = 0; n < 2 * KS; ++n) {
+            o_acc[n][2 * h] *= alpha;
+            o_acc[n][2 * h + 1] *= alpha;
+          }
         }
+        base[h] = (m_run[h] == -INFINITY) ? 0.f : m_run[h];
       }
       float pr[2][4];
 #pragma unroll

@@ -43,6 +43,7 @@ DeviceInfo g_dev[64];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::atomic<int> g_force_path{0};
 std::atomic<int> g_force_tps{0};
+std::atomic<int> g_force_pf_splits{0};
 
 int device_info(DeviceInfo** out) {
   int dev = 0;
@@ -120,7 +121,7 @@ struct Plan {
   int max_tiles = 0;
   long long ctas = 0;
   int dch = 2, d_pad = 128;           // prefill: TMA boxes per tile, padded head_dim
-  int tiles_per_unit = 0, pairs_per_unit = 0, pair_heads = 0;
+  int tiles_per_unit = 0, pairs_per_unit = 0, pair_heads = 0, split_pairs = 0;
   size_t ws_bytes = 0;      // split partials (o_s, lse_s)
   size_t off_lse = 0;
   size_t ticket_bytes = 0;  // split tickets (kept zero between calls)
@@ -208,9 +209,28 @@ int plan_prefill(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
   pl->max_tiles = max_tiles;
   // Too few tile pairs to fill the GPU (multi-token decode shapes): split each
   // pair's key range so that about one item per SM runs; the splits' partials
-  // are merged by the last split to finish.
-  const long long pairs = pl->ctas;
+  // are merged by the last split to finish.  Units with a single row tile use
+  // both q-tile slots for that tile, on adjacent splits (paired items), so
+  // the two softmax warpgroups still alternate.
   pl->splits = 1;
+  pl->split_pairs = 0;
+  const int forced_splits = g_force_pf_splits.load();
+  if (pl->tiles_per_unit == 1 && max_tiles >= 2 && (pr.units < dev.sms || forced_splits > 1)) {
+    long long half = forced_splits > 1 ? (forced_splits + 1) / 2 : dev.sms / pr.units;
+    if (half > (max_tiles + 1) / 2) half = (max_tiles + 1) / 2;
+    if (half < 1) half = 1;
+    pl->split_pairs = 1;
+    pl->splits = (int)(2 * half);
+    pl->pairs_per_unit = 1;
+    pl->ctas = pr.units * half;
+    const size_t tiles = (size_t)pr.units;
+    pl->ws_bytes = align256(tiles * pl->splits * (size_t)pl->d_pad * kPfM * 4);
+    pl->off_lse = pl->ws_bytes;
+    pl->ws_bytes += align256(tiles * pl->splits * 2 * kPfM * 4);
+    pl->ticket_bytes = align256(tiles * 4 * sizeof(unsigned int));
+    return GQA_ATTN_OK;
+  }
+  const long long pairs = pl->ctas;
   if (pairs < dev.sms && max_tiles > 1) {
     long long s = dev.sms / (pairs > 0 ? pairs : 1);
     if (s > max_tiles) s = max_tiles;
@@ -428,6 +448,7 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.tiles_per_unit = pl.tiles_per_unit;
   p.pairs_per_unit = pl.pairs_per_unit;
   p.splits = pl.splits;
+  p.split_pairs = pl.split_pairs;
   p.n_items = (int)pl.ctas;
   p.ws_o = (float*)ws;
   p.ws_ml = ws ? (float*)((char*)ws + pl.off_lse) : nullptr;
@@ -608,6 +629,10 @@ int gqa_attn_set_override(int key, int value) {
   }
   if (key == 2) {
     g_force_tps.store(value > 0 ? value : 0);
+    return GQA_ATTN_OK;
+  }
+  if (key == 3) {
+    g_force_pf_splits.store(value > 0 ? value : 0);
     return GQA_ATTN_OK;
   }
   return GQA_ATTN_ERR_ARG;

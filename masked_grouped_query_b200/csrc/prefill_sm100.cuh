@@ -60,9 +60,11 @@ struct PrefillParams {
   int q_len, kv_len, head_dim, d_pad;
   int rows;              // rows per unit: group * q_len
   int tiles_per_unit;    // ceil(rows / 128)
-  int pairs_per_unit;    // tile pairs per unit
+  int pairs_per_unit;    // tile pairs per unit (row tiles per unit when split_pairs)
   int splits;            // key-range splits per tile pair (1 = none)
-  int n_items;           // units * pairs_per_unit * splits
+  int split_pairs;       // 1: both tiles of an item are the same row tile, taking
+                         // key splits 2s and 2s + 1 (units with one row tile)
+  int n_items;           // units * pairs_per_unit * splits (/ 2 when split_pairs)
   int pair_heads;        // 1: tiles (2p, 2p+1) are two heads at one position
   int causal, window;
   float logit_scale, cap_in, cap_out;
@@ -120,20 +122,50 @@ __device__ __forceinline__ TileInfo prefill_tile(const PrefillParams& p, const M
 }
 
 // One work item: a unit, its pair of q tiles and one split of the union of
-// their key-tile ranges: key tiles [j_first, j_first + j_count).  An item
-// without key tiles is not "busy": no loads or MMAs run for it.
+// their key-tile ranges: key tiles [j_first, j_first + j_count).  With
+// split_pairs both tiles are the same row tile and take adjacent key splits:
+// tile t processes key tiles [kt0[t], kt0[t] + kc[t]), so the two softmax
+// warpgroups still alternate.  An item without key tiles is not "busy": no
+// loads or MMAs run for it.
 struct PfItem {
   int unit;
   int pair_index;  // unit * pairs_per_unit + pair
-  int split;
+  int split;       // split of tile 0 (tile 1 takes split + 1 when paired)
+  bool paired;
   TileInfo tile[2];
   int j_first, j_count;
+  int kt0[2], kc[2];
   bool busy;
 };
 
 __device__ __forceinline__ PfItem prefill_item(const PrefillParams& p, const MaskSpec& ms,
                                                int item) {
   PfItem it;
+  it.paired = p.split_pairs != 0;
+  if (it.paired) {
+    const int half = p.splits / 2;
+    it.split = 2 * (item % half);
+    it.pair_index = item / half;
+    it.unit = it.pair_index / p.pairs_per_unit;
+    const int tile = it.pair_index % p.pairs_per_unit;
+    TileInfo ti;
+    ti.row0 = tile * kPfM;
+    ti.nrows = min(kPfM, p.rows - ti.row0);
+    ti.kr = key_range(ms, ti.row0, ti.nrows, kPfN);
+    it.tile[0] = ti;
+    it.tile[1] = ti;
+    const int per = (ti.kr.t_count + p.splits - 1) / p.splits;
+    for (int t = 0; t < 2; ++t) {
+      const int js = min(ti.kr.t_count, (it.split + t) * per);
+      const int je = min(ti.kr.t_count, js + per);
+      it.kt0[t] = ti.kr.t_first + js;
+      it.kc[t] = je - js;
+    }
+    it.j_first = it.kt0[0];
+    it.j_count = it.kc[0];  // kc[0] >= kc[1]
+    it.busy = it.j_count > 0;
+    return it;
+  }
   it.split = item % p.splits;
   it.pair_index = item / p.splits;
   it.unit = it.pair_index / p.pairs_per_unit;
@@ -158,14 +190,29 @@ __device__ __forceinline__ PfItem prefill_item(const PrefillParams& p, const Mas
     it.j_first += js;
     it.j_count = je - js;
   }
+  it.kt0[0] = it.kt0[1] = it.j_first;
+  it.kc[0] = it.kc[1] = it.j_count;
   it.busy = it.j_count > 0;
   return it;
 }
 
 __device__ __forceinline__ bool tile_active(const PfItem& it, int t, int j) {
+  if (it.paired) return j < (t == 0 ? it.kc[0] : it.kc[1]);
   const KeyRange& kr = t == 0 ? it.tile[0].kr : it.tile[1].kr;
   const int jj = it.j_first + j;
   return kr.t_count > 0 && jj >= kr.t_first && jj < kr.t_first + kr.t_count;
+}
+
+// Key tile that tile t works on at iteration j.
+__device__ __forceinline__ int key_tile(const PfItem& it, int t, int j) {
+  return (t == 0 ? it.kt0[0] : it.kt0[1]) + j;
+}
+
+// Ring position (relative to the item's first load) of K (kv = 0) or V
+// (kv = 1) for tile t at iteration j when paired: each iteration loads K, V
+// of tile 0, then K, V of tile 1 while tile 1 is active.
+__device__ __forceinline__ int paired_pos(const PfItem& it, int t, int j, int kv) {
+  return 2 * j + 2 * min(j, it.kc[1]) + 2 * t + kv;
 }
 
 template <int DCH, bool kCap>
@@ -237,28 +284,35 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!it.busy) continue;
         // The Q buffer is free once every S of the previous busy item is done.
         if (nq > 0 && !(ok = mbar_wait(q_empty, (nq - 1) & 1, kStatusTimeoutProducer))) break;
-        const int ntiles = (it.tile[0].nrows > 0 ? 1 : 0) + (it.tile[1].nrows > 0 ? 1 : 0);
+        // Paired items share tile 0's Q.
+        const int qtiles = it.paired ? 1 : 2;
+        int ntiles = 0;
+        for (int t = 0; t < qtiles; ++t) ntiles += it.tile[t].nrows > 0 ? 1 : 0;
         mbar_arrive_expect_tx(q_full, ntiles * C::kTileBytes);
-        for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < qtiles; ++t)
           if (it.tile[t].nrows > 0)
             for (int c = 0; c < DCH; ++c)
               tma_load_3d(sq + t * C::kTileBytes + c * C::kBoxBytes, &tm_q, q_full, c * 64,
                           it.tile[t].row0, it.unit);
         ++nq;
         for (int j = 0; j < it.j_count && ok; ++j) {
-          const int key0 = (it.j_first + j) * kPfN;
-          for (int kv = 0; kv < 2; ++kv) {
-            const int s = u % C::kSlots;
-            if (u >= C::kSlots &&
-                !(ok = mbar_wait(&kv_empty[s], ((u / C::kSlots) - 1) & 1,
-                                 kStatusTimeoutProducer)))
-              break;
-            uint8_t* dst = ring + s * C::kTileBytes;
-            mbar_arrive_expect_tx(&kv_full[s], C::kTileBytes);
-            for (int c = 0; c < DCH; ++c)
-              tma_load_3d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, &kv_full[s], c * 64, key0,
-                          it.unit);
-            ++u;
+          // One K/V stream per iteration, or one per active tile when paired.
+          const int streams = it.paired ? (tile_active(it, 1, j) ? 2 : 1) : 1;
+          for (int st = 0; st < streams && ok; ++st) {
+            const int key0 = key_tile(it, st, j) * kPfN;
+            for (int kv = 0; kv < 2; ++kv) {
+              const int s = u % C::kSlots;
+              if (u >= C::kSlots &&
+                  !(ok = mbar_wait(&kv_empty[s], ((u / C::kSlots) - 1) & 1,
+                                   kStatusTimeoutProducer)))
+                break;
+              uint8_t* dst = ring + s * C::kTileBytes;
+              mbar_arrive_expect_tx(&kv_full[s], C::kTileBytes);
+              for (int c = 0; c < DCH; ++c)
+                tma_load_3d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, &kv_full[s], c * 64,
+                            key0, it.unit);
+              ++u;
+            }
           }
         }
       }
@@ -295,9 +349,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           return mbar_wait(&kv_full[u % C::kSlots], (u / C::kSlots) & 1, kStatusTimeoutMma);
         };
         auto release = [&](int idx) { mma_commit(&kv_empty[(ubase + idx) % C::kSlots]); };
-        auto issue_s = [&](int t, int j) {
-          const uint32_t kslot = slot_addr(2 * j);
-          const uint32_t qt = sq_addr + t * C::kTileBytes;
+        auto issue_s_at = [&](int t, uint32_t kslot) {
+          const uint32_t qt = sq_addr + (it.paired ? 0 : t * C::kTileBytes);
           const uint32_t d_tmem = tmem + t * 128;
           tc_fence_after();
           for (int ks = 0; ks < ksteps; ++ks) {
@@ -308,8 +361,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           mma_commit(&s_full[t]);
           if (--s_left == 0) mma_commit(q_empty);  // Q no longer read: it may be reloaded
         };
-        auto issue_pv = [&](int t, int j, bool first) {
-          const uint32_t vslot = slot_addr(2 * j + 1);
+        auto issue_pv_at = [&](int t, uint32_t vslot, bool first) {
           const uint32_t p_tmem = tmem + t * 128;
           const uint32_t o_tmem = tmem + 256 + t * 128;
           tc_fence_after();
@@ -318,6 +370,45 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         sdesc_sw128(vslot + ks * 2048, C::kBoxBytes, 1024), idesc_o,
                         (!first || ks > 0) ? 1u : 0u);
         };
+        bool first_pv[2] = {true, true};
+        if (it.paired) {
+          // Each tile has its own K/V stream; every slot is released right
+          // after its only reader is issued.
+          auto pos = [&](int t, int j, int kv) { return paired_pos(it, t, j, kv); };
+          if (!(ok = wait_slot(pos(0, 0, 0)))) break;
+          issue_s_at(0, slot_addr(pos(0, 0, 0)));
+          release(pos(0, 0, 0));
+          for (int j = 0; j < it.j_count && ok; ++j) {
+            for (int t = 0; t < 2 && ok; ++t) {
+              if (!tile_active(it, t, j)) continue;
+              if (!(ok = wait_slot(pos(t, j, 1)))) break;  // V_t(j)
+              if (!(ok = mbar_wait(&p_full[t], n_act[t] & 1, kStatusTimeoutMma))) break;
+              if (j == 0 && t == 0 && tile_active(it, 1, 0)) {  // delayed start of tile B
+                if (!(ok = wait_slot(pos(1, 0, 0)))) break;
+                issue_s_at(1, slot_addr(pos(1, 0, 0)));
+                release(pos(1, 0, 0));
+              }
+              issue_pv_at(t, slot_addr(pos(t, j, 1)), first_pv[t]);
+              first_pv[t] = false;
+              ++n_act[t];
+              release(pos(t, j, 1));
+              if (tile_active(it, t, j + 1)) {
+                if (!(ok = wait_slot(pos(t, j + 1, 0)))) break;
+                issue_s_at(t, slot_addr(pos(t, j + 1, 0)));
+                release(pos(t, j + 1, 0));
+              }
+            }
+          }
+          if (!ok) break;
+          mma_commit(&o_done[0]);
+          mma_commit(&o_done[1]);
+          ubase += paired_pos(it, 0, it.j_count, 0);
+          continue;
+        }
+        auto issue_s = [&](int t, int j) { issue_s_at(t, slot_addr(2 * j)); };
+        auto issue_pv = [&](int t, int j, bool first) {
+          issue_pv_at(t, slot_addr(2 * j + 1), first);
+        };
 
         // Prologue: S(0) of the first active tile only; the other tile's S(0)
         // follows once the first tile's P(0) is ready.
@@ -325,7 +416,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const bool both0 = tile_active(it, 0, 0) && tile_active(it, 1, 0);
         if (tile_active(it, 0, 0)) issue_s(0, 0);
         else if (tile_active(it, 1, 0)) issue_s(1, 0);
-        bool first_pv[2] = {true, true};
         for (int j = 0; j < it.j_count && ok; ++j) {
           if (!(ok = wait_slot(2 * j + 1))) break;  // V_j
           bool k_next_ready = j + 1 >= it.j_count;
@@ -390,7 +480,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       int act = 0;  // key tiles this q tile consumed in this item
       for (int j = 0; j < it.j_count && ok; ++j) {
         if (!tile_active(it, t, j)) continue;
-        const int jj = it.j_first + j;
+        const int jj = key_tile(it, t, j);
         ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], n_act & 1, kStatusTimeoutSoftmax));
         if (!ok) break;
         tc_fence_after();
@@ -412,31 +502,38 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const bool need_mask = !(key0 >= ti.kr.all_lo && key0 + kPfN - 1 <= ti.kr.all_hi);
         // Softcap: when every |score| of the warp's rows maps to |y| <= 1/2 the
         // tanh runs as a polynomial on the FMA pipe, leaving MUFU to ex2.
+        // Row max of the raw scores (8 chains); scale and softcap are
+        // increasing, so the log2-domain max is the transform of this one.
+        // With a softcap the same pass takes the min: when every |x / s| of
+        // the warp's rows is <= 1/2 the tanh runs as a polynomial on the FMA
+        // pipe, leaving MUFU to ex2.
+        float mx[8], mn[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = mn[i] = x[i];
+#pragma unroll
+        for (int c = 8; c < 128; ++c) {
+          mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+          if constexpr (kCap) mn[c & 7] = fminf(mn[c & 7], x[c]);
+        }
+        float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         bool small_y = false;
         if constexpr (kCap) {
-          float am[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) am[i] = fabsf(x[i]);
-#pragma unroll
-          for (int c = 8; c < 128; ++c) am[c & 7] = fmaxf(am[c & 7], fabsf(x[c]));
-          const float amax = fmaxf(fmaxf(fmaxf(am[0], am[1]), fmaxf(am[2], am[3])),
-                                   fmaxf(fmaxf(am[4], am[5]), fmaxf(am[6], am[7])));
-          small_y = __all_sync(0xffffffffu, amax * p.cap_in <= 0.5f);
+          const float mnr = fminf(fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3])),
+                                  fminf(fminf(mn[4], mn[5]), fminf(mn[6], mn[7])));
+          small_y = __all_sync(0xffffffffu, fmaxf(mraw, -mnr) * p.cap_in <= 0.5f);
         }
         if (need_mask) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (key0 + c < lo || key0 + c > hi) x[c] = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = x[i];
+#pragma unroll
+          for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+          mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         }
-        // Row max of the raw scores (a tree of 8 chains); scale and softcap
-        // are increasing, so the log2-domain max is the transform of this one.
-        float mx[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = x[i];
-#pragma unroll
-        for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-        const float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                 fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
         const float mt = mraw == -INFINITY ? -INFINITY
                          : kCap ? p.cap_out * (small_y ? tanh_poly_small(mraw * p.cap_in)
                                                        : tanh_fast(mraw * p.cap_in))
@@ -468,6 +565,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // p = 2^(logit - base) as bf16 pairs into TMEM over S (P chunk q of 32
         // keys lands in columns [16q, 16q + 16), whose scores are consumed).
         if (!kCap || small_y) {
+          // tanh_poly_small's coefficients with cap_in^(2k+1) * cap_out folded in.
+          const float ci2 = p.cap_in * p.cap_in, cc = p.cap_out * p.cap_in;
+          const float q0 = cc * kTanhC1, q1 = cc * ci2 * kTanhC3;
+          const float q2 = cc * ci2 * ci2 * kTanhC5, q3 = cc * ci2 * ci2 * ci2 * kTanhC7;
           // Common case: fully unrolled over the scores already in registers;
           // on mask tiles the logit of a hidden key is forced to -inf.
           const int clo = lo - key0, chi = hi - key0;  // visible columns
@@ -482,10 +583,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 for (int h = 0; h < 2; ++h) {
                   const int col = 32 * q4 + 2 * c + h;
                   float a;
-                  if constexpr (kCap)
-                    a = fmaf(p.cap_out, tanh_poly_small(x[col] * p.cap_in), -base);
-                  else
+                  if constexpr (kCap) {
+                    // cap_out * tanh(x * cap_in) = x * Q(x^2), Q with the caps folded in
+                    a = fmaf(x[col], fmaf(fmaf(fmaf(q3, x[col] * x[col], q2), x[col] * x[col], q1),
+                                          x[col] * x[col], q0),
+                             -base);
+                  } else {
                     a = fmaf(x[col], p.logit_scale, -base);
+                  }
                   if (masked(col)) a = -INFINITY;
                   pe[h] = ex2(a);
                 }
@@ -584,6 +689,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(ov[e]);
         };
         if (p.splits == 1) {
+          if (quarter * 32 >= ti.nrows) continue;  // no row of this warp exists
           const bool live = have && l_run > 0.f;
           const float inv = live ? 1.0f / l_run : 0.f;
           store_rows([&](int col, float (&v)[16]) {
@@ -596,12 +702,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               for (int e = 0; e < 16; ++e) v[e] = 0.f;
             }
           });
-        } else {
+        } else if (quarter * 32 < ti.nrows) {
           // Split partial: O (unnormalised), m, l of this split; the warp
-          // that finishes a row group's last split merges all of them.
-          const long long blk = (long long)(it.pair_index * 2 + t) * p.splits;
-          float* po = p.ws_o + (blk + it.split) * (long long)p.d_pad * kPfM;
-          float* pml = p.ws_ml + (blk + it.split) * 2 * kPfM;
+          // that finishes a row group's last split merges all of them (row
+          // groups wholly past the tile's rows have nothing to write).
+          // Partial block of this row tile and split (paired items: both tiles
+          // are the same rows, splits it.split and it.split + 1).
+          const int ptile = it.paired ? it.pair_index : it.pair_index * 2 + t;
+          const int psplit = it.paired ? it.split + t : it.split;
+          const long long blk = (long long)ptile * p.splits;
+          float* po = p.ws_o + (blk + psplit) * (long long)p.d_pad * kPfM;
+          float* pml = p.ws_ml + (blk + psplit) * 2 * kPfM;
           for (int c0 = 0; c0 < p.d_pad && have; c0 += 16) {
             float v[16];
             load_o(c0, v);
@@ -613,7 +724,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           __threadfence();
           __syncwarp();
           unsigned int ticket = 0;
-          unsigned int* tk = p.tickets + (it.pair_index * 2 + t) * 4 + quarter;
+          unsigned int* tk = p.tickets + ptile * 4 + quarter;
           if (lane == 0) ticket = atomicAdd(tk, 1u);
           ticket = __shfl_sync(0xffffffffu, ticket, 0);
           if (ticket == (unsigned)p.splits - 1) {
@@ -631,13 +742,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             store_rows([&](int col, float (&v)[16]) {
 #pragma unroll
               for (int e = 0; e < 16; ++e) v[e] = 0.f;
-              for (int sp = 0; sp < p.splits; ++sp) {
-                const float m = __ldcg(p.ws_ml + (blk + sp) * 2 * kPfM + r);
-                if (m == -INFINITY) continue;  // empty split: its O was never written
-                const float w = ex2(m - M) * inv;
-                const float* src = p.ws_o + (blk + sp) * (long long)p.d_pad * kPfM + r;
+              // Four splits per batch, all their loads in flight together.
+              for (int sp0 = 0; sp0 < p.splits; sp0 += 4) {
+                float w[4];
+                float x4[4][16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] += w * __ldcg(src + (long long)(col + e) * kPfM);
+                for (int i = 0; i < 4; ++i) {
+                  const int sp = sp0 + i;
+                  const float m = sp < p.splits ? __ldcg(p.ws_ml + (blk + sp) * 2 * kPfM + r)
+                                                : -INFINITY;
+                  // empty split (m = -inf): its O was never written
+                  w[i] = m == -INFINITY ? 0.f : ex2(m - M) * inv;
+                  const float* src =
+                      p.ws_o + (blk + (sp < p.splits ? sp : 0)) * (long long)p.d_pad * kPfM + r;
+#pragma unroll
+                  for (int e = 0; e < 16; ++e)
+                    x4[i][e] = w[i] != 0.f ? __ldcg(src + (long long)(col + e) * kPfM) : 0.f;
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+#pragma unroll
+                  for (int e = 0; e < 16; ++e) v[e] += w[i] * x4[i][e];
               }
             });
             if (lane == 0) atomicExch(tk, 0u);  // ready for the next call

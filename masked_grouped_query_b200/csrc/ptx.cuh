@@ -274,22 +274,16 @@ __device__ __forceinline__ float tanh_fast(float x) {
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-// tanh from its definition, tanh|y| = 1 - 2 / (e^{2|y|} + 1), with the
-// hardware base-2 exponential and reciprocal; absolute error ~1e-7.
-__device__ __forceinline__ float tanh_accurate(float y) {
-  const float a = fabsf(y);
-  const float e = ex2(a * 2.8853900817779268f);  // 2 * log2(e)
-  const float t = 1.0f - 2.0f * rcp(e + 1.0f);
-  return copysignf(t, y);
-}
 // tanh(y) for |y| <= 1/2 on the FMA pipe: y * P(y^2) with a cubic P fitted
 // for least maximum absolute error on [0, 1/2] (1.7e-7; fit_tanh_poly.py
-// next to this file).  Outside that range use tanh_fast / tanh_accurate.
+// next to this file).  Outside that range use tanh_fast.
+constexpr float kTanhC1 = 0.9999978542327881f;
+constexpr float kTanhC3 = -0.3332125246524811f;
+constexpr float kTanhC5 = 0.13148456811904907f;
+constexpr float kTanhC7 = -0.04341723769903183f;
 __device__ __forceinline__ float tanh_poly_small(float y) {
   const float y2 = y * y;
-  return y * fmaf(fmaf(fmaf(-0.04341723769903183f, y2, 0.13148456811904907f), y2,
-                       -0.3332125246524811f),
-                  y2, 0.9999978542327881f);
+  return y * fmaf(fmaf(fmaf(kTanhC7, y2, kTanhC5), y2, kTanhC3), y2, kTanhC1);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {

@@ -190,6 +190,8 @@ def test_forced_split_geometries_agree_with_oracle(tps):
     (2, 20, 3000, 8, 2, 128, True, None, None),     # 80 rows per kv head
     (1, 3, 1000, 16, 1, 72, False, 300, None),      # window without causal, D = 72
     (3, 2, 777, 32, 2, 64, True, None, 20.0),       # ragged keys, D = 64
+    (1, 130, 4000, 2, 1, 128, True, None, 30.0),    # 3 row tiles: two-tile pairs, split
+    (1, 700, 2500, 1, 1, 96, False, 900, None),     # 6 row tiles, window, D = 96
 ])
 def test_tcgen05_key_splits(cfg):
     # Few row tiles: the tcgen05 kernel splits each tile pair's key range
