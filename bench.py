@@ -38,7 +38,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from masked_grouped_query_b200.inputs import WORKLOADS, Workload, make_inputs  # noqa: E402
+from masked_grouped_query_b200.inputs import (CACHE_STEPS, WORKLOADS, CacheStep,  # noqa: E402
+                                              Workload, make_inputs)
 
 DEFAULT_WORKLOAD = "gqa_decode"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -177,13 +178,9 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ native arm
-def time_native(w: Workload, steps: int, warmup: int, device, dist_ctx):
-    import masked_grouped_query_b200 as mgq
-    from masked_grouped_query_b200 import _lib
-
-    lib = _lib.load()
-    q, k, v = (t.to(device) for t in make_inputs(w))
-    out = torch.empty_like(q)
+def _timed_loop(call, steps: int, warmup: int, device, dist_ctx):
+    """Run ``call`` warmup + steps times with an L2 flush before each; time
+    each timed call with CUDA events on the current stream."""
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     sink = torch.empty((), dtype=torch.float32, device=device)
 
@@ -195,19 +192,6 @@ def time_native(w: Workload, steps: int, warmup: int, device, dist_ctx):
         torch.sum(flush, dim=0, out=sink)
 
     stream = torch.cuda.current_stream(device)
-    sh = torch.cuda.current_stream(device).cuda_stream
-    causal, window, cap = int(w.causal), int(w.window or 0), float(w.softcap or 0.0)
-    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), w.batch, w.q_len,
-            w.kv_len, w.num_q_heads, w.num_kv_heads, w.head_dim, causal, window, cap)
-
-    import ctypes
-    sp = ctypes.c_void_p(sh)
-
-    def call():
-        rc = lib.gqa_attn_fwd(*args, sp)
-        if rc != 0:
-            raise RuntimeError(f"gqa_attn_fwd: {_lib.error_string(rc)}")
-
     for _ in range(warmup):
         flush_l2()
         call()
@@ -225,13 +209,95 @@ def time_native(w: Workload, steps: int, warmup: int, device, dist_ctx):
     torch.cuda.synchronize(device)
     wall = time.perf_counter() - t0
     dist_ctx.barrier()
-    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = float(np.mean(per))
-    plan = mgq.describe(w.batch, w.q_len, w.kv_len, w.num_q_heads, w.num_kv_heads,
-                        w.head_dim, w.causal, w.window, w.softcap)
-    return {"ms_mean": ms, "ms_median": float(np.median(per)), "ms_p10": float(np.percentile(per, 10)),
-            "ms_p90": float(np.percentile(per, 90)), "wall_s": wall, "launches": steps,
-            "plan": plan, "status": mgq.status()}
+    per = [st.elapsed_time(en) for st, en in zip(starts, ends)]
+    return {"ms_mean": float(np.mean(per)), "ms_median": float(np.median(per)),
+            "ms_p10": float(np.percentile(per, 10)), "ms_p90": float(np.percentile(per, 90)),
+            "wall_s": wall}
+
+
+def time_native(w: Workload, steps: int, warmup: int, device, dist_ctx):
+    import ctypes
+
+    import masked_grouped_query_b200 as mgq
+    from masked_grouped_query_b200 import _lib
+
+    lib = _lib.load()
+    q, k, v = (t.to(device) for t in make_inputs(w))
+    out = torch.empty_like(q)
+    sp = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    causal, window, cap = int(w.causal), int(w.window or 0), float(w.softcap or 0.0)
+    args = (q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), w.batch, w.q_len,
+            w.kv_len, w.num_q_heads, w.num_kv_heads, w.head_dim, causal, window, cap)
+
+    def call():
+        rc = lib.gqa_attn_fwd(*args, sp)
+        if rc != 0:
+            raise RuntimeError(f"gqa_attn_fwd: {_lib.error_string(rc)}")
+
+    res = _timed_loop(call, steps, warmup, device, dist_ctx)
+    res["launches"] = steps
+    res["plan"] = mgq.describe(w.batch, w.q_len, w.kv_len, w.num_q_heads, w.num_kv_heads,
+                               w.head_dim, w.causal, w.window, w.softcap)
+    res["status"] = mgq.status()
+    return res
+
+
+def time_cache_step(st: CacheStep, steps: int, warmup: int, device, dist_ctx):
+    """One decode step on a (batch, slots, heads, head_dim) bf16 cache: the
+    fp32 new token is appended at ``position`` and attended with the rest,
+    through ``gqa_attn_decode_append``.  Bytes: the attention's K/V union
+    plus the append's fp32 reads and bf16 writes."""
+    import ctypes
+
+    from masked_grouped_query_b200 import _lib
+    from masked_grouped_query_b200.inputs import make_cache_inputs
+
+    lib = _lib.load()
+    x = make_cache_inputs(st.batch, st.slots, st.num_kv_heads, st.head_dim, st.count,
+                          seed=st.seed, num_q_heads=st.num_q_heads, device=device)
+    out = torch.empty_like(x["q"])
+    sp = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    args = (x["q"].data_ptr(), x["k_cache"].data_ptr(), x["v_cache"].data_ptr(),
+            x["new_k"].data_ptr(), x["new_v"].data_ptr(), out.data_ptr(), st.batch, st.count,
+            st.position, st.slots, st.num_q_heads, st.num_kv_heads, st.head_dim,
+            0x1, int(st.causal), int(st.window or 0), float(st.softcap or 0.0), sp)
+
+    def call():
+        rc = lib.gqa_attn_decode_append(*args)
+        if rc != 0:
+            raise RuntimeError(f"gqa_attn_decode_append: {_lib.error_string(rc)}")
+
+    res = _timed_loop(call, steps, warmup, device, dist_ctx)
+    w = Workload(st.name, st.batch, st.count, st.kv_len, st.num_q_heads, st.num_kv_heads,
+                 st.head_dim, st.causal, st.window, st.softcap, st.seed)
+    append_bytes = 2.0 * st.batch * st.count * st.num_kv_heads * st.head_dim * (4 + 2)
+    res["bytes"] = kv_bytes(w) + append_bytes
+    return res
+
+
+def time_kv_append(batch: int, count: int, heads: int, head_dim: int, slots: int, steps: int,
+                   warmup: int, device):
+    """The append kernel alone on a prompt-sized block (fp32 tokens into a
+    bf16 (batch, slots, heads, head_dim) cache): bytes read + written."""
+    import ctypes
+
+    from masked_grouped_query_b200 import _lib
+    from masked_grouped_query_b200.inputs import make_cache_inputs
+
+    lib = _lib.load()
+    x = make_cache_inputs(batch, slots, heads, head_dim, count, seed=17, device=device)
+    sp = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    args = (x["k_cache"].data_ptr(), x["v_cache"].data_ptr(), x["new_k"].data_ptr(),
+            x["new_v"].data_ptr(), batch, slots, heads, head_dim, 0, count, 0x1, None, sp)
+
+    def call():
+        rc = lib.gqa_attn_kv_append(*args)
+        if rc != 0:
+            raise RuntimeError(f"gqa_attn_kv_append: {_lib.error_string(rc)}")
+
+    res = _timed_loop(call, steps, warmup, device, _NoDist())
+    res["bytes"] = 2.0 * batch * count * heads * head_dim * (4 + 2)
+    return res
 
 
 def time_e2e(w: Workload, steps: int, warmup: int, device):
@@ -415,6 +481,18 @@ def main():
             pkv = pk["hbm_gbs"] if u2 == "GB/s" else pk["bf16_tflops"]
             extra[other.name] = {"metric": n2, "value": a, "unit": u2, "ms": r["ms_mean"],
                                  "frac_of_peak": a / pkv, "plan": r["plan"]}
+        for st in CACHE_STEPS.values():
+            r = time_cache_step(st, max(20, args.steps // 4), args.warmup, device, _NoDist())
+            a = r["bytes"] / 1e9 / (r["ms_mean"] * 1e-3)
+            extra[st.name] = {"metric": "decode step on a KV cache (append + attend) GB/s",
+                              "value": a, "unit": "GB/s", "ms": r["ms_mean"],
+                              "frac_of_peak": a / pk["hbm_gbs"], "launches_per_step": 2}
+        r = time_kv_append(2, 4096, 4, 128, 4096, max(20, args.steps // 4), args.warmup, device)
+        a = r["bytes"] / 1e9 / (r["ms_mean"] * 1e-3)
+        extra["kv_append_prompt_block"] = {
+            "metric": "KV-cache append GB/s (fp32 in, bf16 cache, read + written bytes)",
+            "value": a, "unit": "GB/s", "ms": r["ms_mean"], "frac_of_peak": a / pk["hbm_gbs"],
+            "shape": "batch 2, 4096 tokens, 4 kv heads, head_dim 128, (B,S,H,D) cache"}
 
     if ctx.rank == 0:
         if unit == "GB/s":

@@ -197,6 +197,62 @@ int gqa_attn_fwd_static_scratch(const void* q, const void* k, const void* v, voi
                                 int head_dim, int causal, int window, float softcap,
                                 void* stream);
 
+/* ---------------------------------------------------------- KV cache append
+ * Flags for gqa_attn_kv_append and gqa_attn_decode_append (bitwise or). */
+#define GQA_KV_CACHE_SEQ_MAJOR 0x1u /* caches [batch][slots][kv_heads][d]; else [batch][kv_heads][slots][d] */
+#define GQA_KV_CACHE_F32 0x2u       /* caches hold fp32; else bf16 */
+#define GQA_KV_NEW_BF16 0x4u        /* new keys/values are bf16; else fp32 */
+#define GQA_KV_NEW_HEAD_MAJOR 0x8u  /* new keys/values [batch][kv_heads][count][d]; else [batch][count][kv_heads][d] */
+
+/*
+ * Write the keys and values of `count` new tokens into a key cache and a
+ * value cache at slots [position, position + count) ("KV Cache Update at a
+ * Position", TensorTonic, problem statement and constraints): in every batch
+ * row and kv head, slot position + l receives new token l, converted to the
+ * cache dtype (fp32 -> bf16 rounds to nearest even; bf16 -> fp32 is exact);
+ * every other slot keeps its contents.  *new_length (a host int; may be
+ * NULL) receives position + count, the page's returned `length`.
+ *
+ * Layouts (dense, row-major, device memory, 16-byte aligned): the caches are
+ * [batch][cache_slots][num_kv_heads][head_dim] with GQA_KV_CACHE_SEQ_MAJOR
+ * (the page's layout) and [batch][num_kv_heads][cache_slots][head_dim]
+ * without it (the layout gqa_attn_fwd reads); the new keys and values are
+ * [batch][count][num_kv_heads][head_dim] (the page's) or, with
+ * GQA_KV_NEW_HEAD_MAJOR, [batch][num_kv_heads][count][head_dim].  The caller
+ * owns every buffer; the call allocates nothing and is asynchronous on
+ * `stream` (a cudaStream_t; NULL = legacy default stream).
+ *
+ * Errors (nothing is launched): GQA_ATTN_ERR_ARG for unknown flags or
+ * position < 0 or position + count > cache_slots; GQA_ATTN_ERR_BAD_SHAPE,
+ * GQA_ATTN_ERR_HEAD_DIM, GQA_ATTN_ERR_NULL_POINTER, GQA_ATTN_ERR_MISALIGNED
+ * as for gqa_attn_fwd; GQA_ATTN_ERR_ALIAS if the two caches overlap or a new
+ * buffer overlaps a cache.  count == 0 (or batch == 0) launches nothing.
+ */
+int gqa_attn_kv_append(void* k_cache, void* v_cache, const void* new_k, const void* new_v,
+                       int batch, int cache_slots, int num_kv_heads, int head_dim, int position,
+                       int count, unsigned int flags, int* new_length, void* stream);
+
+/*
+ * One decode step on a KV cache: append the q_len new tokens' keys and
+ * values at `position` (gqa_attn_kv_append with the same flags), then
+ * attend q -- the same q_len tokens -- to cache slots [0, position + q_len)
+ * exactly as gqa_attn_fwd with kv_len = position + q_len, so query i sits at
+ * position + i.  Both steps run in order on `stream`; the attention reads
+ * the caches in place, in either layout, with no copy.
+ *
+ * The caches must be bf16 (GQA_KV_CACHE_F32 returns GQA_ATTN_ERR_ARG).  q
+ * and o are [batch][num_q_heads][q_len][head_dim] bf16.  Return codes are
+ * those of both calls; GQA_ATTN_ERR_ALIAS also when q overlaps a cache or o
+ * overlaps a cache, q or a new buffer.  The output equals, bit for bit,
+ * gqa_attn_fwd on contiguous copies of the caches' first position + q_len
+ * slots.
+ */
+int gqa_attn_decode_append(const void* q, void* k_cache, void* v_cache, const void* new_k,
+                           const void* new_v, void* o, int batch, int q_len, int position,
+                           int cache_slots, int num_q_heads, int num_kv_heads, int head_dim,
+                           unsigned int flags, int causal, int window, float softcap,
+                           void* stream);
+
 /* Library version as major * 10000 + minor * 100 + patch. */
 int gqa_attn_version(void);
 

@@ -19,6 +19,7 @@ EXPORTS = (
     "gqa_attn_set_override", "gqa_attn_error_string", "gqa_attn_status",
     "gqa_attn_clear_status", "gqa_attn_selftest_bounded_wait",
     "gqa_attn_version", "gqa_attn_last_error_detail", "gqa_attn_fwd_static_scratch",
+    "gqa_attn_kv_append", "gqa_attn_decode_append",
 )
 
 _I = ctypes.c_int
@@ -75,6 +76,12 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.gqa_attn_last_error_detail.argtypes = []
         lib.gqa_attn_fwd_static_scratch.restype = _I
         lib.gqa_attn_fwd_static_scratch.argtypes = [_P, _P, _P, _P] + _DIMS + [_P]
+        lib.gqa_attn_kv_append.restype = _I
+        lib.gqa_attn_kv_append.argtypes = ([_P] * 4 + [_I] * 6 +
+                                           [ctypes.c_uint, ctypes.POINTER(_I), _P])
+        lib.gqa_attn_decode_append.restype = _I
+        lib.gqa_attn_decode_append.argtypes = ([_P] * 6 + [_I] * 7 +
+                                               [ctypes.c_uint, _I, _I, _F, _P])
         if path is None:
             _lib = lib
         return lib

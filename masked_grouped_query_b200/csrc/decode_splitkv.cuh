@@ -31,6 +31,7 @@ struct DecodeParams {
   const __nv_bfloat16* q;
   __nv_bfloat16* o;
   int q_len, kv_len, head_dim;
+  int kv_heads;        // K/V maps are 4-D: (col, key, kv head, batch)
   int rows;            // rows per (b, kvh): group * q_len
   int row_blocks;      // ceil(rows / 64)
   int block_rows;      // min(64, rows): row stride of the partial buffers
@@ -106,6 +107,7 @@ __global__ void __maxnreg__(kT ? 128 : 255)
     if (lane == 0 && n_tiles > 0) {
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
+      const int kvh = (int)(unit % p.kv_heads), bidx = (int)(unit / p.kv_heads);
       int issued = 0;
       for (int t = 0; t < n_tiles; ++t) {
         const int s = t % C::kStages;
@@ -118,8 +120,8 @@ __global__ void __maxnreg__(kT ? 128 : 255)
         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
 #pragma unroll
         for (int c = 0; c < C::kDChunks; ++c) {
-          tma_load_3d(kt + c * C::kBoxBytes, &tm_k, &full[s], c * 64, key0, unit);
-          tma_load_3d(vt + c * C::kBoxBytes, &tm_v, &full[s], c * 64, key0, unit);
+          tma_load_4d(kt + c * C::kBoxBytes, &tm_k, &full[s], c * 64, key0, kvh, bidx);
+          tma_load_4d(vt + c * C::kBoxBytes, &tm_v, &full[s], c * 64, key0, kvh, bidx);
         }
         ++issued;
       }

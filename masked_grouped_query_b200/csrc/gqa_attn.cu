@@ -21,6 +21,7 @@
 #include "mask.cuh"
 #include "decode_splitkv.cuh"
 #include "prefill_sm100.cuh"
+#include "kv_append.cuh"
 #include "selftest.cuh"
 
 namespace {
@@ -80,6 +81,8 @@ struct Problem {
   int group;
   long long units;  // batch * hkv
   long long rows;   // group * q_len  (rows per unit)
+  long long kv_alloc;  // key slots allocated per (batch, kv head): kv_len, or a cache's slots
+  int kv_seq_major;    // 0: k/v [batch][hkv][kv_alloc][d]; 1: [batch][kv_alloc][hkv][d]
 };
 
 int validate(int batch, int q_len, int kv_len, int hq, int hkv, int d, int causal, int window,
@@ -100,6 +103,8 @@ int validate(int batch, int q_len, int kv_len, int hq, int hkv, int d, int causa
   pr->group = hq / hkv;
   pr->units = (long long)batch * hkv;
   pr->rows = (long long)pr->group * q_len;
+  pr->kv_alloc = kv_len;
+  pr->kv_seq_major = 0;
   // Index limits: element offsets are 64-bit, rows per unit and TMA
   // coordinates are 32-bit, the flattened grid is < 2^31.
   const long long q_elems = (long long)batch * hq * (long long)q_len * d;
@@ -324,6 +329,35 @@ int get_workspace(cudaStream_t stream, size_t bytes, size_t ticket_bytes, void**
 }
 
 // ------------------------------------------------------------------ TMA maps
+// 4-D bf16 view of K or V: (col < d, key < kv_len, kv head, batch) over
+// either cache layout, with a (64 cols x box_rows x 1 x 1) box, 128-byte
+// swizzle; keys at or past kv_len read as zero.
+int encode_kv_map(CUtensorMap* map, const void* base, const Problem& pr, int box_rows) {
+  const cuuint64_t e = 2, d = (cuuint64_t)pr.d, h = (cuuint64_t)pr.hkv,
+                   s = (cuuint64_t)pr.kv_alloc;
+  cuuint64_t dims[4] = {d, (cuuint64_t)pr.kv_len, h, (cuuint64_t)pr.batch};
+  cuuint64_t strides[3];
+  if (pr.kv_seq_major) {
+    strides[0] = h * d * e;      // next key
+    strides[1] = d * e;          // next head
+  } else {
+    strides[0] = d * e;
+    strides[1] = s * d * e;
+  }
+  strides[2] = s * h * d * e;    // next batch element
+  cuuint32_t box[4] = {64, (cuuint32_t)box_rows, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(g_detail, sizeof g_detail, "cuTensorMapEncodeTiled (k/v): CUresult %d", (int)r);
+    return GQA_ATTN_ERR_LAUNCH;
+  }
+  return GQA_ATTN_OK;
+}
+
 // 3-D bf16 view [outer][rows][cols] with a (64 cols x box_rows x 1) box,
 // 128-byte swizzle; out-of-range elements read as zero.
 int encode_map(CUtensorMap* map, const void* base, int cols, long long rows, long long outer,
@@ -362,14 +396,15 @@ int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
     dev.decode_attr[slot] = true;
   }
   CUtensorMap tk, tv;
-  if (encode_map(&tk, k, pr.d, pr.kv_len, pr.units, kDecTile) != GQA_ATTN_OK ||
-      encode_map(&tv, v, pr.d, pr.kv_len, pr.units, kDecTile) != GQA_ATTN_OK)
+  if (encode_kv_map(&tk, k, pr, kDecTile) != GQA_ATTN_OK ||
+      encode_kv_map(&tv, v, pr, kDecTile) != GQA_ATTN_OK)
     return GQA_ATTN_ERR_LAUNCH;
   DecodeParams p;
   p.q = (const __nv_bfloat16*)q;
   p.o = (__nv_bfloat16*)o;
   p.q_len = pr.q_len;
   p.kv_len = pr.kv_len;
+  p.kv_heads = pr.hkv;
   p.head_dim = pr.d;
   p.rows = (int)pr.rows;
   p.row_blocks = pl.row_blocks;
@@ -435,13 +470,14 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   CUtensorMap tq, tk, tv, to;
   if (encode_map(&tq, q, pr.d, pr.rows, pr.units, kPfM) != GQA_ATTN_OK ||
       encode_map(&to, o, pr.d, pr.rows, pr.units, 32) != GQA_ATTN_OK ||
-      encode_map(&tk, k, pr.d, pr.kv_len, pr.units, kPfN) != GQA_ATTN_OK ||
-      encode_map(&tv, v, pr.d, pr.kv_len, pr.units, kPfN) != GQA_ATTN_OK)
+      encode_kv_map(&tk, k, pr, kPfN) != GQA_ATTN_OK ||
+      encode_kv_map(&tv, v, pr, kPfN) != GQA_ATTN_OK)
     return GQA_ATTN_ERR_LAUNCH;
   PrefillParams p;
   p.o = (__nv_bfloat16*)o;
   p.q_len = pr.q_len;
   p.kv_len = pr.kv_len;
+  p.kv_heads = pr.hkv;
   p.head_dim = pr.d;
   p.d_pad = pl.d_pad;
   p.rows = (int)pr.rows;
@@ -487,7 +523,7 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
 int check_pointers(const Problem& pr, const void* q, const void* k, const void* v,
                    const void* o) {
   const size_t q_bytes = (size_t)pr.batch * pr.hq * (size_t)pr.q_len * pr.d * 2;
-  const size_t kv_bytes = (size_t)pr.batch * pr.hkv * (size_t)pr.kv_len * pr.d * 2;
+  const size_t kv_bytes = (size_t)pr.batch * pr.hkv * (size_t)pr.kv_alloc * pr.d * 2;
   if (q_bytes && (!q || !o)) return GQA_ATTN_ERR_NULL_POINTER;
   if (kv_bytes && (!k || !v)) return GQA_ATTN_ERR_NULL_POINTER;
   if (((uintptr_t)q | (uintptr_t)k | (uintptr_t)v | (uintptr_t)o) & 15u)
@@ -679,7 +715,96 @@ int gqa_attn_selftest_bounded_wait(int limit_us, void* stream) {
   return cudaGetLastError() == cudaSuccess ? GQA_ATTN_OK : GQA_ATTN_ERR_LAUNCH;
 }
 
-int gqa_attn_version(void) { return 100; }
+int gqa_attn_version(void) { return 200; }
+
+int gqa_attn_kv_append(void* k_cache, void* v_cache, const void* new_k, const void* new_v,
+                       int batch, int cache_slots, int num_kv_heads, int head_dim, int position,
+                       int count, unsigned int flags, int* new_length, void* stream) {
+  if (flags & ~(GQA_KV_CACHE_SEQ_MAJOR | GQA_KV_CACHE_F32 | GQA_KV_NEW_BF16 |
+                GQA_KV_NEW_HEAD_MAJOR))
+    return GQA_ATTN_ERR_ARG;
+  if (batch < 0 || num_kv_heads < 1 || cache_slots < 0 || count < 0)
+    return GQA_ATTN_ERR_BAD_SHAPE;
+  if (head_dim < 8 || head_dim > 256 || head_dim % 8 != 0) return GQA_ATTN_ERR_HEAD_DIM;
+  if (position < 0 || (long long)position + count > cache_slots) return GQA_ATTN_ERR_ARG;
+  const long long n = (long long)batch * num_kv_heads * count * head_dim;
+  if (new_length) *new_length = position + count;
+  if (n == 0) return GQA_ATTN_OK;
+  if (2 * n / 8 + 4LL * 8 * 1024 * 256 >= (1LL << 32)) {  // chunk indices are 32-bit
+    snprintf(g_detail, sizeof g_detail, "kv_append: %lld new elements exceed the 32-bit index",
+             n);
+    return GQA_ATTN_ERR_TOO_LARGE;
+  }
+  if (!k_cache || !v_cache || !new_k || !new_v) return GQA_ATTN_ERR_NULL_POINTER;
+  if (((uintptr_t)k_cache | (uintptr_t)v_cache | (uintptr_t)new_k | (uintptr_t)new_v) & 15u)
+    return GQA_ATTN_ERR_MISALIGNED;
+  const size_t cache_bytes = (size_t)batch * num_kv_heads * (size_t)cache_slots * head_dim *
+                             ((flags & GQA_KV_CACHE_F32) ? 4 : 2);
+  const size_t new_bytes = (size_t)n * ((flags & GQA_KV_NEW_BF16) ? 2 : 4);
+  if (overlaps(k_cache, cache_bytes, v_cache, cache_bytes) ||
+      overlaps(new_k, new_bytes, k_cache, cache_bytes) ||
+      overlaps(new_k, new_bytes, v_cache, cache_bytes) ||
+      overlaps(new_v, new_bytes, k_cache, cache_bytes) ||
+      overlaps(new_v, new_bytes, v_cache, cache_bytes))
+    return GQA_ATTN_ERR_ALIAS;
+  DeviceInfo* dev = nullptr;
+  int rc = device_info(&dev);
+  if (rc != GQA_ATTN_OK) return rc;
+  KvAppendParams p;
+  p.k_cache = k_cache;
+  p.v_cache = v_cache;
+  p.new_k = new_k;
+  p.new_v = new_v;
+  p.batch = batch;
+  p.heads = num_kv_heads;
+  p.slots = cache_slots;
+  p.head_dim = head_dim;
+  p.position = position;
+  p.count = count;
+  p.cache_seq_major = (flags & GQA_KV_CACHE_SEQ_MAJOR) ? 1 : 0;
+  p.new_head_major = (flags & GQA_KV_NEW_HEAD_MAJOR) ? 1 : 0;
+  const long long chunks = 2 * n / 8;  // 8 elements per thread, keys then values
+  long long blocks = (chunks + 255) / 256;
+  if (blocks > 8LL * dev->sms) blocks = 8LL * dev->sms;
+  cudaStream_t st = (cudaStream_t)stream;
+  const bool nf = !(flags & GQA_KV_NEW_BF16), cf = (flags & GQA_KV_CACHE_F32) != 0;
+  if (nf && cf) kv_append_kernel<true, true><<<(unsigned)blocks, 256, 0, st>>>(p);
+  else if (nf) kv_append_kernel<true, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+  else if (cf) kv_append_kernel<false, true><<<(unsigned)blocks, 256, 0, st>>>(p);
+  else kv_append_kernel<false, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? GQA_ATTN_OK : cuda_fail("launch(kv_append)", e, GQA_ATTN_ERR_LAUNCH);
+}
+
+int gqa_attn_decode_append(const void* q, void* k_cache, void* v_cache, const void* new_k,
+                           const void* new_v, void* o, int batch, int q_len, int position,
+                           int cache_slots, int num_q_heads, int num_kv_heads, int head_dim,
+                           unsigned int flags, int causal, int window, float softcap,
+                           void* stream) {
+  if (flags & GQA_KV_CACHE_F32) return GQA_ATTN_ERR_ARG;  // attention reads bf16 caches
+  if (position < 0 || cache_slots < 0 || (long long)position + q_len > cache_slots)
+    return GQA_ATTN_ERR_ARG;
+  Problem pr;
+  int rc = validate(batch, q_len, position + q_len, num_q_heads, num_kv_heads, head_dim, causal,
+                    window, softcap, &pr);
+  if (rc != GQA_ATTN_OK) return rc;
+  pr.kv_alloc = cache_slots;
+  pr.kv_seq_major = (flags & GQA_KV_CACHE_SEQ_MAJOR) ? 1 : 0;
+  rc = check_pointers(pr, q, k_cache, v_cache, o);
+  if (rc != GQA_ATTN_OK) return rc;
+  const size_t o_bytes = (size_t)batch * num_q_heads * (size_t)q_len * head_dim * 2;
+  const size_t new_bytes = (size_t)batch * num_kv_heads * (size_t)q_len * head_dim *
+                           ((flags & GQA_KV_NEW_BF16) ? 2 : 4);
+  const size_t q_bytes = o_bytes, cache_bytes = (size_t)batch * num_kv_heads *
+                                                  (size_t)cache_slots * head_dim * 2;
+  if (overlaps(o, o_bytes, new_k, new_bytes) || overlaps(o, o_bytes, new_v, new_bytes) ||
+      overlaps(q, q_bytes, k_cache, cache_bytes) || overlaps(q, q_bytes, v_cache, cache_bytes))
+    return GQA_ATTN_ERR_ALIAS;
+  rc = gqa_attn_kv_append(k_cache, v_cache, new_k, new_v, batch, cache_slots, num_kv_heads,
+                          head_dim, position, q_len, flags, nullptr, stream);
+  if (rc != GQA_ATTN_OK) return rc;
+  return run(pr, q, k_cache, v_cache, o, (cudaStream_t)stream);
+}
 
 const char* gqa_attn_last_error_detail(void) { return g_detail; }
 

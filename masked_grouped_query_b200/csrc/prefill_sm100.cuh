@@ -58,6 +58,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 struct PrefillParams {
   __nv_bfloat16* o;
   int q_len, kv_len, head_dim, d_pad;
+  int kv_heads;          // K/V maps are 4-D: (col, key, kv head, batch)
   int rows;              // rows per unit: group * q_len
   int tiles_per_unit;    // ceil(rows / 128)
   int pairs_per_unit;    // tile pairs per unit (row tiles per unit when split_pairs)
@@ -300,6 +301,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const int streams = it.paired ? (tile_active(it, 1, j) ? 2 : 1) : 1;
           for (int st = 0; st < streams && ok; ++st) {
             const int key0 = key_tile(it, st, j) * kPfN;
+            const int kvh = it.unit % p.kv_heads, bidx = it.unit / p.kv_heads;
             for (int kv = 0; kv < 2; ++kv) {
               const int s = u % C::kSlots;
               if (u >= C::kSlots &&
@@ -309,8 +311,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               uint8_t* dst = ring + s * C::kTileBytes;
               mbar_arrive_expect_tx(&kv_full[s], C::kTileBytes);
               for (int c = 0; c < DCH; ++c)
-                tma_load_3d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, &kv_full[s], c * 64,
-                            key0, it.unit);
+                tma_load_4d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, &kv_full[s], c * 64,
+                            key0, kvh, bidx);
               ++u;
             }
           }

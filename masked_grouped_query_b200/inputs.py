@@ -102,3 +102,63 @@ def make_inputs_device(w: Workload, device, seed: int | None = None):
     k = torch.randn(ks, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
     v = torch.randn(ks, generator=g, device=device, dtype=torch.float32).to(torch.bfloat16)
     return q, k, v
+
+
+@dataclass(frozen=True)
+class CacheStep:
+    """One decode step on a KV cache: ``count`` new tokens appended at
+    ``position`` into caches of ``slots`` slots, then attended by the same
+    tokens' queries over slots [0, position + count)."""
+
+    name: str
+    batch: int
+    slots: int
+    position: int
+    count: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    causal: bool
+    window: int | None
+    softcap: float | None
+    seed: int
+
+    @property
+    def kv_len(self) -> int:
+        return self.position + self.count
+
+
+# The grouped-query decode shape above, run on a cache in the KV-cache page's
+# (batch, slots, heads, head_dim) layout: the 8192th token is appended and
+# attends to all 8192 slots.
+CACHE_STEPS = {
+    "gqa_decode_append": CacheStep(
+        "gqa_decode_append", 16, 8192, 8191, 1, 32, 8, 128, True, None, None, 5),
+}
+
+
+def make_cache_inputs(batch: int, slots: int, heads: int, head_dim: int, count: int, *,
+                      cache_dtype=torch.bfloat16, new_dtype=torch.float32, seed: int = 0,
+                      num_q_heads: int | None = None, device="cpu"):
+    """Seeded caches and new tokens in the KV-cache page's layouts.
+
+    Returns a dict with k_cache, v_cache (batch, slots, heads, head_dim) in
+    ``cache_dtype``; new_k, new_v (batch, count, heads, head_dim) in
+    ``new_dtype`` (fp32 on the page); and, when ``num_q_heads`` is given, q
+    (batch, num_q_heads, count, head_dim) bf16.  Standard-normal draws in the
+    order k_cache, v_cache, new_k, new_v, q.
+    """
+    gen_dev = "cpu" if str(device) == "cpu" else device
+    g = torch.Generator(device=gen_dev).manual_seed(seed)
+
+    def draw(shape, dtype):
+        x = torch.randn(shape, generator=g, device=device, dtype=torch.float32)
+        return x if dtype == torch.float32 else x.to(dtype)
+
+    cs = (batch, slots, heads, head_dim)
+    ns = (batch, count, heads, head_dim)
+    out = dict(k_cache=draw(cs, cache_dtype), v_cache=draw(cs, cache_dtype),
+               new_k=draw(ns, new_dtype), new_v=draw(ns, new_dtype))
+    if num_q_heads is not None:
+        out["q"] = draw((batch, num_q_heads, count, head_dim), torch.bfloat16)
+    return out

@@ -71,11 +71,50 @@ def test_rejects_bad_pointers_without_a_device(lib):
     assert _fwd(lib, dims=big) == -10
 
 
+def _append(lib, kc=0x1000, vc=0x100000, nk=0x200000, nv=0x300000, b=1, s=8, h=2, d=64,
+            pos=0, n=1, flags=0):
+    P = ctypes.c_void_p
+    return lib.gqa_attn_kv_append(P(kc), P(vc), P(nk), P(nv), b, s, h, d, pos, n, flags,
+                                  None, None)
+
+
+def test_append_rejects_bad_arguments_without_a_device(lib):
+    assert _append(lib, pos=-1) == -12
+    assert _append(lib, pos=8) == -12            # 8 + 1 > 8 slots
+    assert _append(lib, pos=5, n=4) == -12
+    assert _append(lib, flags=0x10) == -12       # unknown flag
+    assert _append(lib, d=60) == -5
+    assert _append(lib, h=0) == -3
+    assert _append(lib, kc=0) == -1
+    assert _append(lib, nk=0x200008) == -2
+    assert _append(lib, vc=0x1000 + 64) == -11   # caches overlap
+    assert _append(lib, nk=0x1000 + 512) == -11  # new keys inside the key cache
+    assert _append(lib, n=0, kc=0) == 0          # nothing to write: no device needed
+    length = ctypes.c_int(-1)
+    P = ctypes.c_void_p
+    assert lib.gqa_attn_kv_append(P(0), P(0), P(0), P(0), 1, 8, 2, 64, 3, 0, 0,
+                                  ctypes.byref(length), None) == 0
+    assert length.value == 3
+    # the decode step takes bf16 caches only, and checks the block fits
+    q = o = None
+    assert lib.gqa_attn_decode_append(P(0x10000), P(0x20000), P(0x80000), P(0x100000),
+                                      P(0x110000), P(0x120000), 1, 1, 7, 8, 4, 2, 64, 0x2,
+                                      1, 0, 0.0, None) == -12
+    assert lib.gqa_attn_decode_append(P(0x10000), P(0x20000), P(0x80000), P(0x100000),
+                                      P(0x110000), P(0x120000), 1, 2, 7, 8, 4, 2, 64, 0,
+                                      1, 0, 0.0, None) == -12
+    assert lib.gqa_attn_decode_append(P(0x20000), P(0x20000), P(0x80000), P(0x100000),
+                                      P(0x110000), P(0x120000), 1, 1, 7, 8, 4, 2, 64, 0,
+                                      1, 0, 0.0, None) == -11   # q inside the key cache
+    del q, o
+
+
 def test_no_device_means_device_error(lib):
     if torch.cuda.is_available():
         pytest.skip("a CUDA device is present")
     assert _fwd(lib) == -7
     assert lib.gqa_attn_selftest_bounded_wait(100, None) == -7
+    assert _append(lib) == -7
 
 
 def test_empty_problem_is_a_no_op(lib):
