@@ -231,8 +231,10 @@ int plan_prefill(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
     const size_t tiles = (size_t)pr.units;
     pl->ws_bytes = align256(tiles * pl->splits * (size_t)pl->d_pad * kPfM * 4);
     pl->off_lse = pl->ws_bytes;
-    pl->ws_bytes += align256(tiles * pl->splits * 2 * kPfM * 4);
-    pl->ticket_bytes = align256(tiles * 4 * sizeof(unsigned int));
+    // (m, l) per split, per column half of the softmax, per row
+    pl->ws_bytes += align256(tiles * pl->splits * 2 * 2 * kPfM * 4);
+    // one ticket per (tile, lane quarter, column half)
+    pl->ticket_bytes = align256(tiles * 8 * sizeof(unsigned int));
     return GQA_ATTN_OK;
   }
   const long long pairs = pl->ctas;
@@ -246,8 +248,8 @@ int plan_prefill(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
   if (pl->splits > 1) {
     pl->ws_bytes = align256((size_t)pairs * 2 * pl->splits * (size_t)pl->d_pad * kPfM * 4);
     pl->off_lse = pl->ws_bytes;
-    pl->ws_bytes += align256((size_t)pairs * 2 * pl->splits * 2 * kPfM * 4);
-    pl->ticket_bytes = align256((size_t)pairs * 2 * 4 * sizeof(unsigned int));
+    pl->ws_bytes += align256((size_t)pairs * 2 * pl->splits * 2 * 2 * kPfM * 4);
+    pl->ticket_bytes = align256((size_t)pairs * 2 * 8 * sizeof(unsigned int));
   }
   return GQA_ATTN_OK;
 }

@@ -23,15 +23,20 @@
 //               O_t += P_t V_j (A = P from TMEM, B = V from shared memory,
 //               N = head_dim rounded up to 16);
 //   warps 2-3   idle (they complete warpgroup 0 for the register split);
-//   warps 4-7   softmax + epilogue for tile A, warps 8-11 for tile B: one
-//               thread per row reads its S row from TMEM, applies scale,
-//               softcap and mask, keeps the running max / sum in fp32
-//               (online softmax, rescaling O in TMEM only when the max grows
-//               by more than 2^8), writes P as bf16 back over S in TMEM, and
-//               at the end of the item normalises O and stores its bf16 row.
-// Tile B's first S is issued only once tile A's first P is ready, so the two
-// softmax warpgroups run out of phase: while one computes its softmax the
-// tensor core works on the other tile's P.V and next S.
+//   warps 4-11  softmax + epilogue: warps 4-7 take key columns [0, 64) of
+//               each S tile, warps 8-11 columns [64, 128).  A thread owns
+//               half of one row: it reads that half from TMEM, applies
+//               scale, softcap and mask, and swaps its partial row max with
+//               the partner thread (same TMEM lane, other half) through
+//               shared memory under a named barrier; both then keep the same
+//               running max (online softmax, rescaling their halves of O in
+//               TMEM only when the max grows by more than 2^8), write P as
+//               bf16 back over S in TMEM and keep half-row sums, added up at
+//               the end of the item, when each half normalises and stores
+//               its half of the O row.
+// The eight softmax warps take tile A, then tile B, at every key step: while
+// they work on one tile the tensor core runs the other tile's P.V and next
+// S, and two warps per SM sub-partition share each softmax.
 //
 // Fully masked key tiles are never loaded; tiles wholly inside every row's
 // visible range skip the per-element mask.  All waits are bounded.
@@ -86,7 +91,9 @@ struct PrefillCfg {
   static constexpr int kRingBytes = kSlots * kTileBytes;
   // Output staging: one 32-row x 64-column bf16 box (4 KB) per softmax warp.
   static constexpr int kStageBytes = 8 * 4096;
-  static constexpr int kBarOffset = kQBytes + kRingBytes + kStageBytes;
+  // Row values swapped between the two column halves: [half][row] fp32.
+  static constexpr int kXchgBytes = 2 * 128 * 4;
+  static constexpr int kBarOffset = kQBytes + kRingBytes + kStageBytes + kXchgBytes;
   // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain
   static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 1;
   static constexpr int kSmemBytes = 1024 + kBarOffset + kNumBars * 8 + 16;
@@ -228,6 +235,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint8_t* sq = smem;                   // Q tiles A, B
   uint8_t* ring = smem + C::kQBytes;    // K/V slots
   uint8_t* stage_all = ring + C::kRingBytes;  // output staging, 4 KB per softmax warp
+  float* xchg = (float*)(stage_all + C::kStageBytes);
   uint64_t* bars = (uint64_t*)(smem + C::kBarOffset);
   uint64_t* q_full = bars;
   uint64_t* q_empty = bars + 1;
@@ -251,7 +259,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
+      mbar_init(&p_full[t], 256);
       mbar_init(&o_done[t], 1);
     }
     mbar_init(drain, 1);
@@ -380,16 +388,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (!(ok = wait_slot(pos(0, 0, 0)))) break;
           issue_s_at(0, slot_addr(pos(0, 0, 0)));
           release(pos(0, 0, 0));
+          if (tile_active(it, 1, 0)) {
+            if (!(ok = wait_slot(pos(1, 0, 0)))) break;
+            issue_s_at(1, slot_addr(pos(1, 0, 0)));
+            release(pos(1, 0, 0));
+          }
           for (int j = 0; j < it.j_count && ok; ++j) {
             for (int t = 0; t < 2 && ok; ++t) {
               if (!tile_active(it, t, j)) continue;
               if (!(ok = wait_slot(pos(t, j, 1)))) break;  // V_t(j)
               if (!(ok = mbar_wait(&p_full[t], n_act[t] & 1, kStatusTimeoutMma))) break;
-              if (j == 0 && t == 0 && tile_active(it, 1, 0)) {  // delayed start of tile B
-                if (!(ok = wait_slot(pos(1, 0, 0)))) break;
-                issue_s_at(1, slot_addr(pos(1, 0, 0)));
-                release(pos(1, 0, 0));
-              }
               issue_pv_at(t, slot_addr(pos(t, j, 1)), first_pv[t]);
               first_pv[t] = false;
               ++n_act[t];
@@ -412,19 +420,16 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           issue_pv_at(t, slot_addr(2 * j + 1), first);
         };
 
-        // Prologue: S(0) of the first active tile only; the other tile's S(0)
-        // follows once the first tile's P(0) is ready.
+        // Prologue: S(0) of both tiles; the softmax takes tile A, then B.
         if (!(ok = wait_slot(0))) break;
-        const bool both0 = tile_active(it, 0, 0) && tile_active(it, 1, 0);
         if (tile_active(it, 0, 0)) issue_s(0, 0);
-        else if (tile_active(it, 1, 0)) issue_s(1, 0);
+        if (tile_active(it, 1, 0)) issue_s(1, 0);
         for (int j = 0; j < it.j_count && ok; ++j) {
           if (!(ok = wait_slot(2 * j + 1))) break;  // V_j
           bool k_next_ready = j + 1 >= it.j_count;
           for (int t = 0; t < 2 && ok; ++t) {
             if (tile_active(it, t, j)) {
               if (!(ok = mbar_wait(&p_full[t], n_act[t] & 1, kStatusTimeoutMma))) break;
-              if (j == 0 && t == 0 && both0) issue_s(1, 0);  // delayed start of tile B
               issue_pv(t, j, first_pv[t]);
               first_pv[t] = false;
               ++n_act[t];
@@ -458,230 +463,271 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax / epilogue
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
-    const int t = (warp - 4) / 4;            // tile 0 (A) or 1 (B)
+    // Warps 4-7 take key columns [0, 64) of every S tile, warps 8-11 columns
+    // [64, 128).  Warps w and w + 4 read the same TMEM lane quarter (w & 3),
+    // i.e. the same 32 rows: partner threads own the two halves of one row
+    // and swap row values through `xchg` under named barrier 1 + quarter.
+    // All eight warps process tile A, then tile B, at every key step.
+    const int h = (warp - 4) / 4;            // column half
     const int quarter = warp & 3;            // TMEM lane quarter of this warp
-    const int r = quarter * 32 + lane;       // row within the tile
+    const int r = quarter * 32 + lane;       // row within a q tile
+    const int bar_id = 1 + quarter;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const uint32_t s_tmem = tmem + lane_base + t * 128;
-    const uint32_t o_tmem = tmem + lane_base + 256 + t * 128;
-    int n_act = 0;   // S tiles consumed (s_full phases)
-    int n_done = 0;  // busy items finished (o_done phases)
+    const int oc0 = min(64 * h, p.d_pad), oc1 = min(64 * h + 64, p.d_pad);  // O columns
+    uint8_t* stage = stage_all + (warp - 4) * 4096;
+    // Swap `mine` with the partner's value; `okv` becomes the AND over the
+    // pair.  The first barrier guarantees the partner has read the previous
+    // value before it is overwritten; the fences order TMEM accesses of the
+    // two threads around the barriers.
+    auto exchange = [&](float mine, bool& okv) -> float {
+      tc_fence_before();
+      named_bar_sync(bar_id, 64);
+      xchg[h * kPfM + r] = mine;
+      okv = named_bar_and(bar_id, 64, okv);
+      tc_fence_after();
+      return xchg[(1 - h) * kPfM + r];
+    };
+    struct RowState {
+      int lo, hi;       // visible keys of this thread's row (hi < lo: none)
+      int act;          // key tiles consumed in this item
+      float m, l;       // running max (log2 domain) and this half's running sum
+    };
+    int n_act0 = 0, n_act1 = 0;  // S tiles consumed per q tile (s_full phases)
+    int n_done = 0;              // busy items finished (o_done phases)
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const PfItem it = prefill_item(p, ms, item);
-      const TileInfo ti = t == 0 ? it.tile[0] : it.tile[1];
-      const long long grow = (long long)ti.row0 + r;  // row within the unit
-      const bool row_valid = r < ti.nrows;
-      int lo = 0, hi = -1;
-      if (row_valid) {
-        const int qpos = p.kv_len - p.q_len + (int)(grow % p.q_len);
-        lo = first_key(ms, qpos);
-        hi = last_key(ms, qpos);
+      RowState st[2];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        st[t].lo = 0;
+        st[t].hi = -1;
+        st[t].act = 0;
+        st[t].m = -INFINITY;
+        st[t].l = 0.f;
+        if (r < it.tile[t].nrows) {
+          const long long grow = (long long)it.tile[t].row0 + r;  // row within the unit
+          const int qpos = p.kv_len - p.q_len + (int)(grow % p.q_len);
+          st[t].lo = first_key(ms, qpos);
+          st[t].hi = last_key(ms, qpos);
+        }
       }
-      float m_run = -INFINITY, l_run = 0.f;
-      int act = 0;  // key tiles this q tile consumed in this item
       for (int j = 0; j < it.j_count && ok; ++j) {
-        if (!tile_active(it, t, j)) continue;
-        const int jj = key_tile(it, t, j);
-        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], n_act & 1, kStatusTimeoutSoftmax));
-        if (!ok) break;
-        tc_fence_after();
-        uint32_t s0[32], s1[32], s2[32], s3[32];
-        tmem_ld32(s_tmem + 0, s0);
-        tmem_ld32(s_tmem + 32, s1);
-        tmem_ld32(s_tmem + 64, s2);
-        tmem_ld32(s_tmem + 96, s3);
-        tmem_ld_wait();
-        float x[128];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = __uint_as_float(s0[c]);
-          x[32 + c] = __uint_as_float(s1[c]);
-          x[64 + c] = __uint_as_float(s2[c]);
-          x[96 + c] = __uint_as_float(s3[c]);
-        }
-        const int key0 = jj * kPfN;
-        const bool need_mask = !(key0 >= ti.kr.all_lo && key0 + kPfN - 1 <= ti.kr.all_hi);
-        // Softcap: when every |score| of the warp's rows maps to |y| <= 1/2 the
-        // tanh runs as a polynomial on the FMA pipe, leaving MUFU to ex2.
-        // Row max of the raw scores (8 chains); scale and softcap are
-        // increasing, so the log2-domain max is the transform of this one.
-        // With a softcap the same pass takes the min: when every |x / s| of
-        // the warp's rows is <= 1/2 the tanh runs as a polynomial on the FMA
-        // pipe, leaving MUFU to ex2.
-        float mx[8], mn[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = mn[i] = x[i];
-#pragma unroll
-        for (int c = 8; c < 128; ++c) {
-          mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-          if constexpr (kCap) mn[c & 7] = fminf(mn[c & 7], x[c]);
-        }
-        float mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-        bool small_y = false;
-        if constexpr (kCap) {
-          const float mnr = fminf(fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3])),
-                                  fminf(fminf(mn[4], mn[5]), fminf(mn[6], mn[7])));
-          small_y = __all_sync(0xffffffffu, fmaxf(mraw, -mnr) * p.cap_in <= 0.5f);
-        }
-        if (need_mask) {
-#pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (key0 + c < lo || key0 + c > hi) x[c] = -INFINITY;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) mx[i] = x[i];
-#pragma unroll
-          for (int c = 8; c < 128; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-          mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-        }
-        const float mt = mraw == -INFINITY ? -INFINITY
-                         : kCap ? p.cap_out * (small_y ? tanh_poly_small(mraw * p.cap_in)
-                                                       : tanh_fast(mraw * p.cap_in))
-                                : mraw * p.logit_scale;
-        // Rescale only when the max grew by more than 2^8 (or was -inf): the
-        // stale max keeps p <= 256, and O / l stays consistent either way.
-        const float m_new = fmaxf(m_run, mt);
-        const bool need =
-            (m_new > m_run + kRescaleThreshold) || (m_run == -INFINITY && m_new != -INFINITY);
-        const float alpha = need ? ex2(m_run - m_new) : 1.0f;  // 0 when m_run = -inf
-        if (need) {
-          l_run *= alpha;
-          m_run = m_new;
-        }
-        if (__any_sync(0xffffffffu, need) && act > 0) {
-          // tcgen05.ld/st are warp-collective: every lane takes part.
-          for (int c0 = 0; c0 < p.d_pad; c0 += 16) {
-            uint32_t ov[16];
-            tmem_ld16(o_tmem + c0, ov);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!tile_active(it, t, j)) continue;
+          // One body for both tiles: the tile's state moves into `cs`.
+          RowState cs = t ? st[1] : st[0];
+          const KeyRange kr = t ? it.tile[1].kr : it.tile[0].kr;
+          const int nph = t ? n_act1 : n_act0;
+          const uint32_t s_tmem = tmem + lane_base + t * 128 + 64 * h;
+          const uint32_t o_tmem = tmem + lane_base + 256 + t * 128;
+          const int ktile0 = key_tile(it, t, j) * kPfN;
+          const int key0 = ktile0 + 64 * h;  // key of this half's column 0
+          const bool need_mask = !(ktile0 >= kr.all_lo && ktile0 + kPfN - 1 <= kr.all_hi);
+          const int clo = cs.lo - key0, chi = cs.hi - key0;  // visible columns
+          bool wok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], nph & 1, kStatusTimeoutSoftmax));
+          float x[64];
+          float mraw = -INFINITY;
+          bool small_y = false;
+          if (wok) {
+            tc_fence_after();
+            uint32_t s0[32], s1[32];
+            tmem_ld32(s_tmem + 0, s0);
+            tmem_ld32(s_tmem + 32, s1);
             tmem_ld_wait();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st16(o_tmem + c0, ov);
-          }
-          tmem_st_wait();
-        }
-        const float base = m_run == -INFINITY ? 0.f : m_run;
-        float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        // p = 2^(logit - base) as bf16 pairs into TMEM over S (P chunk q of 32
-        // keys lands in columns [16q, 16q + 16), whose scores are consumed).
-        if (!kCap || small_y) {
-          // tanh_poly_small's coefficients with cap_in^(2k+1) * cap_out folded in.
-          const float ci2 = p.cap_in * p.cap_in, cc = p.cap_out * p.cap_in;
-          const float q0 = cc * kTanhC1, q1 = cc * ci2 * kTanhC3;
-          const float q2 = cc * ci2 * ci2 * kTanhC5, q3 = cc * ci2 * ci2 * ci2 * kTanhC7;
-          // Common case: fully unrolled over the scores already in registers;
-          // on mask tiles the logit of a hidden key is forced to -inf.
-          const int clo = lo - key0, chi = hi - key0;  // visible columns
-          auto emit = [&](auto masked) {
+            for (int c = 0; c < 32; ++c) {
+              x[c] = __uint_as_float(s0[c]);
+              x[32 + c] = __uint_as_float(s1[c]);
+            }
+            // Softcap: when every |x / s| of the warp's columns is <= 1/2 the
+            // tanh runs as a polynomial on the FMA pipe, leaving MUFU to ex2;
+            // the min of the raw scores (before masking) decides it.
+            if constexpr (kCap) {
+              float mx[8], mn[8];
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4) {
+              for (int i = 0; i < 8; ++i) mx[i] = mn[i] = x[i];
+#pragma unroll
+              for (int c = 8; c < 64; ++c) {
+                mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+                mn[c & 7] = fminf(mn[c & 7], x[c]);
+              }
+              mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+              const float mnr = fminf(fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3])),
+                                      fminf(fminf(mn[4], mn[5]), fminf(mn[6], mn[7])));
+              small_y = __all_sync(0xffffffffu, fmaxf(mraw, -mnr) * p.cap_in <= 0.5f);
+            }
+            if (!kCap || need_mask) {
+              // Row max of the raw scores over visible keys (8 chains); scale
+              // and softcap are increasing, so the log2-domain max is the
+              // transform of this one.
+              if (need_mask) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                  if (c < clo || c > chi) x[c] = -INFINITY;
+              }
+              float mx[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) mx[i] = x[i];
+#pragma unroll
+              for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+              mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            }
+          }
+          const float mrow = fmaxf(mraw, exchange(mraw, wok));
+          if (!wok) {
+            ok = false;
+            break;
+          }
+          // The same transform of the same value in both halves: the row's
+          // max is bitwise equal in the two partner threads.
+          const float mt = mrow == -INFINITY ? -INFINITY
+                           : kCap ? p.cap_out * tanh_fast(mrow * p.cap_in)
+                                  : mrow * p.logit_scale;
+          // Rescale only when the max grew by more than 2^8 (or was -inf):
+          // the stale max keeps p <= 256, and O / l stays consistent.
+          const float m_new = fmaxf(cs.m, mt);
+          const bool need =
+              (m_new > cs.m + kRescaleThreshold) || (cs.m == -INFINITY && m_new != -INFINITY);
+          const float alpha = need ? ex2(cs.m - m_new) : 1.0f;  // 0 when m = -inf
+          if (need) {
+            cs.l *= alpha;
+            cs.m = m_new;
+          }
+          if (__any_sync(0xffffffffu, need) && cs.act > 0) {
+            // This half's O columns; tcgen05.ld/st are warp-collective.
+            for (int c0 = oc0; c0 < oc1; c0 += 16) {
+              uint32_t ov[16];
+              tmem_ld16(o_tmem + c0, ov);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 16; ++e)
+                ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+              tmem_st16(o_tmem + c0, ov);
+            }
+            tmem_st_wait();
+          }
+          const float base = cs.m == -INFINITY ? 0.f : cs.m;
+          float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+          // p = 2^(logit - base) as bf16 pairs into TMEM over S: the 32 keys of
+          // chunk g of the tile land in columns [16g, 16g + 16).  Both halves
+          // loaded their S before the exchange, so no unread score is
+          // overwritten.  A hidden key (x = -inf) gives p = 0.
+          const uint32_t p_tmem = tmem + lane_base + t * 128 + 32 * h;
+          auto emit = [&](auto logit, auto zero_hidden) {
+#pragma unroll
+            for (int q2 = 0; q2 < 2; ++q2) {
               uint32_t pk[16];
 #pragma unroll
               for (int c = 0; c < 16; ++c) {
                 float pe[2];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                  const int col = 32 * q4 + 2 * c + h;
-                  float a;
-                  if constexpr (kCap) {
-                    // cap_out * tanh(x * cap_in) = x * Q(x^2), Q with the caps folded in
-                    a = fmaf(x[col], fmaf(fmaf(fmaf(q3, x[col] * x[col], q2), x[col] * x[col], q1),
-                                          x[col] * x[col], q0),
-                             -base);
-                  } else {
-                    a = fmaf(x[col], p.logit_scale, -base);
-                  }
-                  if (masked(col)) a = -INFINITY;
-                  pe[h] = ex2(a);
+                for (int e = 0; e < 2; ++e) {
+                  const int col = 32 * q2 + 2 * c + e;
+                  pe[e] = ex2(logit(x[col]));
+                  if (zero_hidden(col)) pe[e] = 0.f;
                 }
                 ls[c & 7] += pe[0] + pe[1];
                 pk[c] = pack_bf16(pe[0], pe[1]);
               }
-              tmem_st16(s_tmem + 16 * q4, pk);
+              tmem_st16(p_tmem + 16 * q2, pk);
             }
           };
-          if (need_mask)
-            emit([&](int col) { return col < clo || col > chi; });
-          else
-            emit([](int) { return false; });
-        } else {
-          // Softcap with large arguments (hardware tanh): a compact loop over
-          // 32 scores at a time re-read from TMEM; hidden keys get p = 0.
-          const int clo = need_mask ? lo - key0 : 0;
-          const int chi = need_mask ? hi - key0 : kPfN - 1;
-#pragma unroll 1
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t sv[32];
-            tmem_ld32(s_tmem + 32 * q4, sv);
-            tmem_ld_wait();
-            uint32_t pk[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              float pe[2];
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int col = 32 * q4 + 2 * c + h;
-                const float a =
-                    fmaf(p.cap_out, tanh_fast(__uint_as_float(sv[2 * c + h]) * p.cap_in), -base);
-                pe[h] = (col < clo || col > chi) ? 0.f : ex2(a);
-              }
-              ls[c & 7] += pe[0] + pe[1];
-              pk[c] = pack_bf16(pe[0], pe[1]);
+          auto none = [](int) { return false; };
+          if constexpr (!kCap) {
+            const float sc = p.logit_scale;
+            emit([&](float v) { return fmaf(v, sc, -base); }, none);
+          } else {
+            // With a softcap a hidden key's logit is not -inf, so its p is
+            // zeroed explicitly.
+            auto hidden = [&](int col) { return x[col] == -INFINITY; };
+            if (small_y) {
+              // tanh_poly_small's coefficients with cap_in^(2k+1) * cap_out
+              // folded in: cap_out * tanh(x * cap_in) = x * Q(x^2).
+              const float ci2 = p.cap_in * p.cap_in, cc = p.cap_out * p.cap_in;
+              const float q0 = cc * kTanhC1, q1 = cc * ci2 * kTanhC3;
+              const float q2c = cc * ci2 * ci2 * kTanhC5, q3 = cc * ci2 * ci2 * ci2 * kTanhC7;
+              auto logit = [&](float v) {
+                const float v2 = v * v;
+                return fmaf(v, fmaf(fmaf(fmaf(q3, v2, q2c), v2, q1), v2, q0), -base);
+              };
+              if (need_mask) emit(logit, hidden);
+              else emit(logit, none);
+            } else {
+              const float co = p.cap_out, ci = p.cap_in;
+              auto logit = [&](float v) { return fmaf(co, tanh_fast(v * ci), -base); };
+              if (need_mask) emit(logit, hidden);
+              else emit(logit, none);
             }
-            tmem_st16(s_tmem + 16 * q4, pk);
+          }
+          cs.l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&p_full[t]);
+          ++cs.act;
+          if (t) {
+            st[1] = cs;
+            ++n_act1;
+          } else {
+            st[0] = cs;
+            ++n_act0;
           }
         }
-        l_run += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
-        tmem_st_wait();
-        tc_fence_before();
-        mbar_arrive(&p_full[t]);
-        ++n_act;
-        ++act;
       }
       if (!ok) break;
-      // ---- epilogue: o = O / l as bf16, one row per thread.  The next item's
-      // first P.V may overwrite O only after this warpgroup's next P arrival,
-      // which follows these (waited) TMEM loads in program order.
+      // ---- epilogue: o = O / l as bf16.  The next item's first P.V may
+      // overwrite O only after the next P arrival of all eight warps, which
+      // follows these (waited) TMEM loads in program order.  One barrier
+      // covers both tiles: every MMA of the item has finished.
+      bool eok = true;
       if (it.busy) {
-        ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], n_done & 1, kStatusTimeoutEpilogue));
+        eok = __all_sync(0xffffffffu, mbar_wait(&o_done[0], n_done & 1, kStatusTimeoutEpilogue));
         ++n_done;
-        if (!ok) break;
-        tc_fence_after();
       }
-      if (ti.nrows > 0) {
-        const bool have = act > 0;
-        uint8_t* stage = stage_all + (t * 4 + quarter) * 4096;
-        // Write this warp's 32 output rows as bf16: through its 128B-swizzled
-        // 32-row staging box, 64 columns at a time, each written out by one
-        // TMA store (rows past the unit's end are not written).  value16(col,
-        // v) fills v with the fp32 outputs of columns col .. col + 15.
-        auto store_rows = [&](auto value16) {
-          for (int c0 = 0; c0 < p.d_pad; c0 += 64) {
-            const int ncols = min(64, p.d_pad - c0);
-            if (lane == 0) bulk_wait_read();  // the previous store has read the box
-            __syncwarp();
-            for (int c1 = 0; c1 < ncols; c1 += 16) {
-              float v[16];
-              value16(c0 + c1, v);
+      // Row sums: the two halves add the same two values in the same order.
+      float lsum[2];
 #pragma unroll
-              for (int g = 0; g < 2; ++g) {  // 8 columns = one 16-byte chunk
-                const uint4 w = make_uint4(pack_bf16(v[8 * g], v[8 * g + 1]),
-                                           pack_bf16(v[8 * g + 2], v[8 * g + 3]),
-                                           pack_bf16(v[8 * g + 4], v[8 * g + 5]),
-                                           pack_bf16(v[8 * g + 6], v[8 * g + 7]));
-                *reinterpret_cast<uint4*>(stage + sw128(lane, (c1 >> 3) + g)) = w;
-              }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_3d(&tm_o, stage, c0, ti.row0 + quarter * 32, it.unit);
-              bulk_commit();
-            }
+      for (int t = 0; t < 2; ++t) {
+        const float other = exchange(st[t].l, eok);
+        lsum[t] = h == 0 ? st[t].l + other : other + st[t].l;
+      }
+      if (!eok) break;
+      tc_fence_after();
+      // Write this warp's 32 rows, columns [oc0, oc1), as bf16 through its
+      // 128B-swizzled 32-row staging box and one TMA store (rows past the
+      // unit's end are not written).  value16(col, v) fills v with the fp32
+      // outputs of columns col .. col + 15.
+      auto store_rows = [&](const TileInfo& ti, auto value16) {
+        if (lane == 0) bulk_wait_read();  // the previous store has read the box
+        __syncwarp();
+        for (int c1 = 0; c1 < oc1 - oc0; c1 += 16) {
+          float v[16];
+          value16(oc0 + c1, v);
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {  // 8 columns = one 16-byte chunk
+            const uint4 w = make_uint4(pack_bf16(v[8 * g], v[8 * g + 1]),
+                                       pack_bf16(v[8 * g + 2], v[8 * g + 3]),
+                                       pack_bf16(v[8 * g + 4], v[8 * g + 5]),
+                                       pack_bf16(v[8 * g + 6], v[8 * g + 7]));
+            *reinterpret_cast<uint4*>(stage + sw128(lane, (c1 >> 3) + g)) = w;
           }
-        };
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&tm_o, stage, oc0, ti.row0 + quarter * 32, it.unit);
+          bulk_commit();
+        }
+      };
+      for (int t = 0; t < 2; ++t) {
+        const TileInfo ti = t ? it.tile[1] : it.tile[0];
+        if (ti.nrows <= 0 || quarter * 32 >= ti.nrows || oc0 >= oc1) continue;
+        const RowState cs = t ? st[1] : st[0];
+        const float L = t ? lsum[1] : lsum[0];
+        const uint32_t o_tmem = tmem + lane_base + 256 + t * 128;
+        const bool have = cs.act > 0;
         // O columns col .. col + 15 of this thread's row from TMEM (warp-collective).
         auto load_o = [&](int col, float (&v)[16]) {
           uint32_t ov[16];
@@ -691,10 +737,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(ov[e]);
         };
         if (p.splits == 1) {
-          if (quarter * 32 >= ti.nrows) continue;  // no row of this warp exists
-          const bool live = have && l_run > 0.f;
-          const float inv = live ? 1.0f / l_run : 0.f;
-          store_rows([&](int col, float (&v)[16]) {
+          const bool live = have && L > 0.f;
+          const float inv = live ? 1.0f / L : 0.f;
+          store_rows(ti, [&](int col, float (&v)[16]) {
             if (have) {
               load_o(col, v);
 #pragma unroll
@@ -704,44 +749,43 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               for (int e = 0; e < 16; ++e) v[e] = 0.f;
             }
           });
-        } else if (quarter * 32 < ti.nrows) {
-          // Split partial: O (unnormalised), m, l of this split; the warp
-          // that finishes a row group's last split merges all of them (row
-          // groups wholly past the tile's rows have nothing to write).
-          // Partial block of this row tile and split (paired items: both tiles
-          // are the same rows, splits it.split and it.split + 1).
+        } else {
+          // Split partial: O (unnormalised, this half's columns), m and l of
+          // this split; the warp that finishes a row group's last split
+          // merges all of them.  Paired items: both tiles are the same rows,
+          // splits it.split and it.split + 1.  m and l are kept per half, so
+          // each half's merge reads only what its own warps wrote.
           const int ptile = it.paired ? it.pair_index : it.pair_index * 2 + t;
           const int psplit = it.paired ? it.split + t : it.split;
           const long long blk = (long long)ptile * p.splits;
           float* po = p.ws_o + (blk + psplit) * (long long)p.d_pad * kPfM;
-          float* pml = p.ws_ml + (blk + psplit) * 2 * kPfM;
-          for (int c0 = 0; c0 < p.d_pad && have; c0 += 16) {
+          auto ml_of = [&](int sp) { return p.ws_ml + ((blk + sp) * 2 + h) * 2 * kPfM; };
+          for (int c0 = oc0; c0 < oc1 && have; c0 += 16) {
             float v[16];
             load_o(c0, v);
 #pragma unroll
             for (int e = 0; e < 16; ++e) po[(long long)(c0 + e) * kPfM + r] = v[e];
           }
-          pml[r] = have ? m_run : -INFINITY;
-          pml[kPfM + r] = have ? l_run : 0.f;
+          float* pml = ml_of(psplit);
+          pml[r] = have ? cs.m : -INFINITY;
+          pml[kPfM + r] = have ? L : 0.f;
           __threadfence();
           __syncwarp();
           unsigned int ticket = 0;
-          unsigned int* tk = p.tickets + ptile * 4 + quarter;
+          unsigned int* tk = p.tickets + (ptile * 4 + quarter) * 2 + h;
           if (lane == 0) ticket = atomicAdd(tk, 1u);
           ticket = __shfl_sync(0xffffffffu, ticket, 0);
           if (ticket == (unsigned)p.splits - 1) {
             __threadfence();
             float M = -INFINITY;
-            for (int sp = 0; sp < p.splits; ++sp)
-              M = fmaxf(M, __ldcg(p.ws_ml + (blk + sp) * 2 * kPfM + r));
-            float L = 0.f;
+            for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, __ldcg(ml_of(sp) + r));
+            float Ls = 0.f;
             for (int sp = 0; sp < p.splits; ++sp) {
-              const float* ml = p.ws_ml + (blk + sp) * 2 * kPfM;
-              const float m = __ldcg(ml + r);
-              L += m == -INFINITY ? 0.f : ex2(m - M) * __ldcg(ml + kPfM + r);
+              const float m = __ldcg(ml_of(sp) + r);
+              Ls += m == -INFINITY ? 0.f : ex2(m - M) * __ldcg(ml_of(sp) + kPfM + r);
             }
-            const float inv = L > 0.f ? 1.0f / L : 0.f;
-            store_rows([&](int col, float (&v)[16]) {
+            const float inv = Ls > 0.f ? 1.0f / Ls : 0.f;
+            store_rows(ti, [&](int col, float (&v)[16]) {
 #pragma unroll
               for (int e = 0; e < 16; ++e) v[e] = 0.f;
               // Four splits per batch, all their loads in flight together.
@@ -751,8 +795,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                   const int sp = sp0 + i;
-                  const float m = sp < p.splits ? __ldcg(p.ws_ml + (blk + sp) * 2 * kPfM + r)
-                                                : -INFINITY;
+                  const float m = sp < p.splits ? __ldcg(ml_of(sp) + r) : -INFINITY;
                   // empty split (m = -inf): its O was never written
                   w[i] = m == -INFINITY ? 0.f : ex2(m - M) * inv;
                   const float* src =
