@@ -420,10 +420,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           issue_pv_at(t, slot_addr(2 * j + 1), first);
         };
 
-        // Prologue: S(0) of both tiles; the softmax takes tile A, then B.
+        // Prologue: S(0) of both tiles (K_0's only readers, so its slot is
+        // released at once); the softmax takes tile A, then B.
         if (!(ok = wait_slot(0))) break;
         if (tile_active(it, 0, 0)) issue_s(0, 0);
         if (tile_active(it, 1, 0)) issue_s(1, 0);
+        release(0);
         for (int j = 0; j < it.j_count && ok; ++j) {
           if (!(ok = wait_slot(2 * j + 1))) break;  // V_j
           bool k_next_ready = j + 1 >= it.j_count;
@@ -445,9 +447,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           // K_{j+1} must have landed before it can be released.
           if (ok && !k_next_ready) ok = wait_slot(2 * (j + 1));
           if (!ok) break;
-          // Release each slot once its last reader is issued: K_0 after both
-          // S(0), V_j after P.V of iteration j, K_{j+1} after S of j+1.
-          if (j == 0) release(0);
+          // Release each slot once its last reader is issued: V_j after P.V
+          // of iteration j, K_{j+1} after S of j+1.
           release(2 * j + 1);
           if (j + 1 < it.j_count) release(2 * (j + 1));
         }
