@@ -38,8 +38,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from masked_grouped_query_b200.inputs import (CACHE_STEPS, WORKLOADS, CacheStep,  # noqa: E402
-                                              Workload, make_inputs)
+from masked_grouped_query_b200.inputs import (CACHE_STEPS, RING_STEPS, WORKLOADS,  # noqa: E402
+                                              CacheStep, Workload, make_inputs)
 
 DEFAULT_WORKLOAD = "gqa_decode"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -275,6 +275,39 @@ def time_cache_step(st: CacheStep, steps: int, warmup: int, device, dist_ctx):
     return res
 
 
+def time_ring(rs: dict, steps: int, warmup: int, device):
+    """gqa_attn_fwd_ring on a (batch, kv_heads, slots, head_dim) ring: bytes
+    are the K/V of the window's keys, read once per kv head."""
+    import ctypes
+
+    from masked_grouped_query_b200 import _lib
+
+    lib = _lib.load()
+    g = torch.Generator(device=device).manual_seed(rs["seed"])
+    ks = (rs["batch"], rs["num_kv_heads"], rs["slots"], rs["head_dim"])
+    kr = torch.randn(ks, generator=g, device=device).bfloat16()
+    vr = torch.randn(ks, generator=g, device=device).bfloat16()
+    q = torch.randn(rs["batch"], rs["num_q_heads"], rs["q_len"], rs["head_dim"], generator=g,
+                    device=device).bfloat16()
+    out = torch.empty_like(q)
+    sp = ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    args = (q.data_ptr(), kr.data_ptr(), vr.data_ptr(), out.data_ptr(), rs["batch"], rs["q_len"],
+            rs["kv_len"], rs["slots"], rs["num_q_heads"], rs["num_kv_heads"], rs["head_dim"], 0,
+            int(rs["causal"]), int(rs["window"] or 0), float(rs["softcap"] or 0.0), sp)
+
+    def call():
+        rc = lib.gqa_attn_fwd_ring(*args)
+        if rc != 0:
+            raise RuntimeError(f"gqa_attn_fwd_ring: {_lib.error_string(rc)}")
+
+    res = _timed_loop(call, steps, warmup, device, _NoDist())
+    w = Workload("ring", rs["batch"], rs["q_len"], rs["kv_len"], rs["num_q_heads"],
+                 rs["num_kv_heads"], rs["head_dim"], rs["causal"], rs["window"], rs["softcap"],
+                 rs["seed"])
+    res["bytes"] = kv_bytes(w)
+    return res
+
+
 def time_kv_append(batch: int, count: int, heads: int, head_dim: int, slots: int, steps: int,
                    warmup: int, device):
     """The append kernel alone on a prompt-sized block (fp32 tokens into a
@@ -487,6 +520,13 @@ def main():
             extra[st.name] = {"metric": "decode step on a KV cache (append + attend) GB/s",
                               "value": a, "unit": "GB/s", "ms": r["ms_mean"],
                               "frac_of_peak": a / pk["hbm_gbs"], "launches_per_step": 2}
+        for name, rs in RING_STEPS.items():
+            r = time_ring(rs, max(20, args.steps // 4), args.warmup, device)
+            a = r["bytes"] / 1e9 / (r["ms_mean"] * 1e-3)
+            extra[name] = {"metric": "masked-GQA attn fwd KV-read GB/s (decode, ring window)",
+                           "value": a, "unit": "GB/s", "ms": r["ms_mean"],
+                           "frac_of_peak": a / pk["hbm_gbs"],
+                           "shape": {k: v for k, v in rs.items() if k != "seed"}}
         r = time_kv_append(2, 4096, 4, 128, 4096, max(20, args.steps // 4), args.warmup, device)
         a = r["bytes"] / 1e9 / (r["ms_mean"] * 1e-3)
         extra["kv_append_prompt_block"] = {

@@ -203,6 +203,7 @@ int gqa_attn_fwd_static_scratch(const void* q, const void* k, const void* v, voi
 #define GQA_KV_CACHE_F32 0x2u       /* caches hold fp32; else bf16 */
 #define GQA_KV_NEW_BF16 0x4u        /* new keys/values are bf16; else fp32 */
 #define GQA_KV_NEW_HEAD_MAJOR 0x8u  /* new keys/values [batch][kv_heads][count][d]; else [batch][count][kv_heads][d] */
+#define GQA_KV_RING 0x10u           /* ring cache: token p goes to slot p % cache_slots (see below) */
 
 /*
  * Write the keys and values of `count` new tokens into a key cache and a
@@ -222,8 +223,14 @@ int gqa_attn_fwd_static_scratch(const void* q, const void* k, const void* v, voi
  * owns every buffer; the call allocates nothing and is asynchronous on
  * `stream` (a cudaStream_t; NULL = legacy default stream).
  *
+ * With GQA_KV_RING the caches are rings (the layouts above with cache_slots
+ * slots): token position + l goes to slot (position + l) % cache_slots, so
+ * position may exceed cache_slots; count must not (the block would
+ * overwrite itself).
+ *
  * Errors (nothing is launched): GQA_ATTN_ERR_ARG for unknown flags or
- * position < 0 or position + count > cache_slots; GQA_ATTN_ERR_BAD_SHAPE,
+ * position < 0 or position + count > cache_slots (ring: count > cache_slots
+ * or position + count > INT_MAX); GQA_ATTN_ERR_BAD_SHAPE,
  * GQA_ATTN_ERR_HEAD_DIM, GQA_ATTN_ERR_NULL_POINTER, GQA_ATTN_ERR_MISALIGNED
  * as for gqa_attn_fwd; GQA_ATTN_ERR_ALIAS if the two caches overlap or a new
  * buffer overlaps a cache.  count == 0 (or batch == 0) launches nothing.
@@ -240,6 +247,10 @@ int gqa_attn_kv_append(void* k_cache, void* v_cache, const void* new_k, const vo
  * position + i.  Both steps run in order on `stream`; the attention reads
  * the caches in place, in either layout, with no copy.
  *
+ * With GQA_KV_RING the caches are rings and the attention is that of
+ * gqa_attn_fwd_ring with kv_len = position + q_len and ring_slots =
+ * cache_slots.
+ *
  * The caches must be bf16 (GQA_KV_CACHE_F32 returns GQA_ATTN_ERR_ARG).  q
  * and o are [batch][num_q_heads][q_len][head_dim] bf16.  Return codes are
  * those of both calls; GQA_ATTN_ERR_ALIAS also when q overlaps a cache or o
@@ -252,6 +263,30 @@ int gqa_attn_decode_append(const void* q, void* k_cache, void* v_cache, const vo
                            int cache_slots, int num_q_heads, int num_kv_heads, int head_dim,
                            unsigned int flags, int causal, int window, float softcap,
                            void* stream);
+
+/*
+ * Masked GQA attention over keys and values kept in ring buffers (decode
+ * over a sliding window stored circularly): key j of the kv_len-key
+ * sequence lives in slot j % ring_slots of k_ring / v_ring, which are
+ * [batch][num_kv_heads][ring_slots][head_dim] bf16, or
+ * [batch][ring_slots][num_kv_heads][head_dim] with GQA_KV_CACHE_SEQ_MAJOR
+ * (the only flag accepted).  The result is that of gqa_attn_fwd on the keys
+ * in order -- same mask rule, query i at kv_len - q_len + i -- provided the
+ * ring still holds every key a query can see: ring_slots >= min(kv_len,
+ * q_len + window - 1) with a window, ring_slots >= kv_len without one.  So a
+ * ring of window + q_len - 1 slots serves a sliding window of `window`.
+ * (Decode rows over ring windows: "CSA2 attention on Metal", TensorFold
+ * pull request 1709, section "What this changes".)
+ *
+ * ring_slots must be a positive multiple of 64.  Computed by the split-KV
+ * decode kernel whatever the number of rows.  Errors: those of
+ * gqa_attn_fwd, and GQA_ATTN_ERR_ARG for a bad ring_slots, a ring too small
+ * for the visible keys (see gqa_attn_last_error_detail) or unknown flags.
+ */
+int gqa_attn_fwd_ring(const void* q, const void* k_ring, const void* v_ring, void* o, int batch,
+                      int q_len, int kv_len, int ring_slots, int num_q_heads, int num_kv_heads,
+                      int head_dim, unsigned int flags, int causal, int window, float softcap,
+                      void* stream);
 
 /* Library version as major * 10000 + minor * 100 + patch. */
 int gqa_attn_version(void);

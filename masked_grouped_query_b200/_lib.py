@@ -19,7 +19,7 @@ EXPORTS = (
     "gqa_attn_set_override", "gqa_attn_error_string", "gqa_attn_status",
     "gqa_attn_clear_status", "gqa_attn_selftest_bounded_wait",
     "gqa_attn_version", "gqa_attn_last_error_detail", "gqa_attn_fwd_static_scratch",
-    "gqa_attn_kv_append", "gqa_attn_decode_append",
+    "gqa_attn_kv_append", "gqa_attn_decode_append", "gqa_attn_fwd_ring",
 )
 
 _I = ctypes.c_int
@@ -82,6 +82,8 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.gqa_attn_decode_append.restype = _I
         lib.gqa_attn_decode_append.argtypes = ([_P] * 6 + [_I] * 7 +
                                                [ctypes.c_uint, _I, _I, _F, _P])
+        lib.gqa_attn_fwd_ring.restype = _I
+        lib.gqa_attn_fwd_ring.argtypes = ([_P] * 4 + [_I] * 7 + [ctypes.c_uint, _I, _I, _F, _P])
         if path is None:
             _lib = lib
         return lib

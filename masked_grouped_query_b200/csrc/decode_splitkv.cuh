@@ -32,6 +32,9 @@ struct DecodeParams {
   __nv_bfloat16* o;
   int q_len, kv_len, head_dim;
   int kv_heads;        // K/V maps are 4-D: (col, key, kv head, batch)
+  int k_base;          // key of tile 0's first column (0, or the ring's key base)
+  int ring_tiles;      // ring: slots / 64 (tile t is in slot tile (ring_phase + t) % ring_tiles); 0: none
+  int ring_phase;
   int rows;            // rows per (b, kvh): group * q_len
   int row_blocks;      // ceil(rows / 64)
   int block_rows;      // min(64, rows): row stride of the partial buffers
@@ -87,7 +90,7 @@ __global__ void __maxnreg__(kT ? 128 : 255)
   const long long r0 = (long long)rb * kDecRows;
   const int nr = min(kDecRows, p.rows - (int)r0);
   const MaskSpec ms{p.q_len, p.kv_len, p.causal, p.window};
-  const KeyRange kr = key_range(ms, r0, nr, kDecTile);
+  const KeyRange kr = key_range_from(ms, r0, nr, kDecTile, p.k_base);
   const int t_begin = split * p.tiles_per_split;
   const int t_end = min(kr.t_count, t_begin + p.tiles_per_split);
   const int n_tiles = max(0, t_end - t_begin);
@@ -116,12 +119,15 @@ __global__ void __maxnreg__(kT ? 128 : 255)
           break;
         uint8_t* kt = ring + s * C::kStageBytes;
         uint8_t* vt = kt + C::kTileBytes;
-        const int key0 = (kr.t_first + t_begin + t) * kDecTile;
+        const int tv = kr.t_first + t_begin + t;
+        // K/V row of the tile: its first key, or its slot tile in a ring.
+        const int row0 = p.ring_tiles ? ((p.ring_phase + tv) % p.ring_tiles) * kDecTile
+                                      : p.k_base + tv * kDecTile;
         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
 #pragma unroll
         for (int c = 0; c < C::kDChunks; ++c) {
-          tma_load_4d(kt + c * C::kBoxBytes, &tm_k, &full[s], c * 64, key0, kvh, bidx);
-          tma_load_4d(vt + c * C::kBoxBytes, &tm_v, &full[s], c * 64, key0, kvh, bidx);
+          tma_load_4d(kt + c * C::kBoxBytes, &tm_k, &full[s], c * 64, row0, kvh, bidx);
+          tma_load_4d(vt + c * C::kBoxBytes, &tm_v, &full[s], c * 64, row0, kvh, bidx);
         }
         ++issued;
       }
@@ -174,7 +180,7 @@ __global__ void __maxnreg__(kT ? 128 : 255)
       if (!mbar_wait(&full[s], (t / C::kStages) & 1, kStatusTimeoutConsumer)) break;
       const uint32_t kbase = smem_u32(ring + s * C::kStageBytes);
       const uint32_t vbase = kbase + C::kTileBytes;
-      const int key0 = (kr.t_first + t_begin + t) * kDecTile;
+      const int key0 = p.k_base + (kr.t_first + t_begin + t) * kDecTile;
       const int wkey0 = wn * 16;
       const bool need_mask = !(key0 >= kr.all_lo && key0 + kDecTile - 1 <= kr.all_hi);
       // ---- S^T = K Q^T (16 keys x 8 rows)
@@ -319,7 +325,7 @@ __global__ void __maxnreg__(kT ? 128 : 255)
     }
     const uint32_t kbase = smem_u32(ring + s * C::kStageBytes);
     const uint32_t vbase = kbase + C::kTileBytes;
-    const int key0 = (kr.t_first + t_begin + t) * kDecTile;
+    const int key0 = p.k_base + (kr.t_first + t_begin + t) * kDecTile;
     const int wkey0 = wn * kw;  // first key of this warp inside the tile
     const bool need_mask = !(key0 >= kr.all_lo && key0 + kDecTile - 1 <= kr.all_hi);
 

@@ -83,6 +83,7 @@ struct Problem {
   long long rows;   // group * q_len  (rows per unit)
   long long kv_alloc;  // key slots allocated per (batch, kv head): kv_len, or a cache's slots
   int kv_seq_major;    // 0: k/v [batch][hkv][kv_alloc][d]; 1: [batch][kv_alloc][hkv][d]
+  int ring;            // ring of `ring` slots (key j in slot j % ring); 0: keys in order
 };
 
 int validate(int batch, int q_len, int kv_len, int hq, int hkv, int d, int causal, int window,
@@ -105,6 +106,7 @@ int validate(int batch, int q_len, int kv_len, int hq, int hkv, int d, int causa
   pr->rows = (long long)pr->group * q_len;
   pr->kv_alloc = kv_len;
   pr->kv_seq_major = 0;
+  pr->ring = 0;
   // Index limits: element offsets are 64-bit, rows per unit and TMA
   // coordinates are 32-bit, the flattened grid is < 2^31.
   const long long q_elems = (long long)batch * hq * (long long)q_len * d;
@@ -150,11 +152,12 @@ int plan_decode(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
   pl->row_blocks = (int)ceil_div(pr.rows, kDecRows);
   pl->block_rows = (int)(pr.rows < kDecRows ? pr.rows : kDecRows);
   const MaskSpec ms{pr.q_len, pr.kv_len, pr.causal, pr.window};
+  const int k_base = pr.ring ? ring_k_base(pr.kv_len, pr.ring, kDecTile) : 0;
   int max_tiles = 0;
   for (int rb = 0; rb < pl->row_blocks; ++rb) {
     const long long r0 = (long long)rb * kDecRows;
     const int nr = (int)((pr.rows - r0) < kDecRows ? (pr.rows - r0) : kDecRows);
-    const KeyRange kr = key_range(ms, r0, nr, kDecTile);
+    const KeyRange kr = key_range_from(ms, r0, nr, kDecTile, k_base);
     if (kr.t_count > max_tiles) max_tiles = kr.t_count;
   }
   pl->max_tiles = max_tiles;
@@ -268,7 +271,8 @@ int make_plan(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
   // 128), with key-range splits when there are few row tiles; the decode
   // kernel also covers head_dim 136..256.
   const int forced = g_force_path.load();
-  const bool prefill_ok = pr.d <= 128;
+  // Ring storage is read by the split-KV kernel only.
+  const bool prefill_ok = pr.d <= 128 && pr.ring == 0;
   bool prefill = pr.rows > 16 && prefill_ok;
   if (forced == 1) prefill = false;
   if (forced == 2 && prefill_ok) prefill = true;
@@ -337,7 +341,9 @@ int get_workspace(cudaStream_t stream, size_t bytes, size_t ticket_bytes, void**
 int encode_kv_map(CUtensorMap* map, const void* base, const Problem& pr, int box_rows) {
   const cuuint64_t e = 2, d = (cuuint64_t)pr.d, h = (cuuint64_t)pr.hkv,
                    s = (cuuint64_t)pr.kv_alloc;
-  cuuint64_t dims[4] = {d, (cuuint64_t)pr.kv_len, h, (cuuint64_t)pr.batch};
+  // A ring's map covers all its slots; keys in order stop at kv_len.
+  const cuuint64_t rows = pr.ring ? (cuuint64_t)pr.ring : (cuuint64_t)pr.kv_len;
+  cuuint64_t dims[4] = {d, rows, h, (cuuint64_t)pr.batch};
   cuuint64_t strides[3];
   if (pr.kv_seq_major) {
     strides[0] = h * d * e;      // next key
@@ -407,6 +413,9 @@ int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.q_len = pr.q_len;
   p.kv_len = pr.kv_len;
   p.kv_heads = pr.hkv;
+  p.k_base = pr.ring ? ring_k_base(pr.kv_len, pr.ring, kDecTile) : 0;
+  p.ring_tiles = pr.ring ? pr.ring / kDecTile : 0;
+  p.ring_phase = pr.ring ? ring_phase(pr.kv_len, pr.ring, kDecTile) : 0;
   p.head_dim = pr.d;
   p.rows = (int)pr.rows;
   p.row_blocks = pl.row_blocks;
@@ -520,6 +529,27 @@ bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
   if (!a || !b || na == 0 || nb == 0) return false;
   const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
   return x < y + nb && y < x + na;
+}
+
+// Ring storage of `slots` slots (key j in slot j % slots): the slots must
+// be whole 64-key tiles and hold every key any query can see, i.e. the
+// keys from kv_len - slots on (the window bounds how far back queries look).
+int set_ring(Problem* pr, int slots) {
+  if (slots <= 0 || slots % kDecTile != 0) return GQA_ATTN_ERR_ARG;
+  long long reach;  // keys back from kv_len that the oldest query may see
+  if (pr->window > 0)
+    reach = (long long)pr->q_len + pr->window - 1;
+  else
+    reach = pr->kv_len;
+  if (reach > pr->kv_len) reach = pr->kv_len;
+  if (reach > slots) {
+    snprintf(g_detail, sizeof g_detail, "ring of %d slots holds fewer keys than the %lld visible",
+             slots, reach);
+    return GQA_ATTN_ERR_ARG;
+  }
+  pr->ring = slots;
+  pr->kv_alloc = slots;
+  return GQA_ATTN_OK;
 }
 
 int check_pointers(const Problem& pr, const void* q, const void* k, const void* v,
@@ -723,12 +753,15 @@ int gqa_attn_kv_append(void* k_cache, void* v_cache, const void* new_k, const vo
                        int batch, int cache_slots, int num_kv_heads, int head_dim, int position,
                        int count, unsigned int flags, int* new_length, void* stream) {
   if (flags & ~(GQA_KV_CACHE_SEQ_MAJOR | GQA_KV_CACHE_F32 | GQA_KV_NEW_BF16 |
-                GQA_KV_NEW_HEAD_MAJOR))
+                GQA_KV_NEW_HEAD_MAJOR | GQA_KV_RING))
     return GQA_ATTN_ERR_ARG;
   if (batch < 0 || num_kv_heads < 1 || cache_slots < 0 || count < 0)
     return GQA_ATTN_ERR_BAD_SHAPE;
   if (head_dim < 8 || head_dim > 256 || head_dim % 8 != 0) return GQA_ATTN_ERR_HEAD_DIM;
-  if (position < 0 || (long long)position + count > cache_slots) return GQA_ATTN_ERR_ARG;
+  const bool ring = (flags & GQA_KV_RING) != 0;
+  if (position < 0 || (long long)position + count > (ring ? 0x7fffffffLL : (long long)cache_slots) ||
+      (ring && count > cache_slots))
+    return GQA_ATTN_ERR_ARG;
   const long long n = (long long)batch * num_kv_heads * count * head_dim;
   if (new_length) *new_length = position + count;
   if (n == 0) return GQA_ATTN_OK;
@@ -765,6 +798,7 @@ int gqa_attn_kv_append(void* k_cache, void* v_cache, const void* new_k, const vo
   p.count = count;
   p.cache_seq_major = (flags & GQA_KV_CACHE_SEQ_MAJOR) ? 1 : 0;
   p.new_head_major = (flags & GQA_KV_NEW_HEAD_MAJOR) ? 1 : 0;
+  p.ring = ring ? 1 : 0;
   const long long chunks = 2 * n / 8;  // 8 elements per thread, keys then values
   long long blocks = (chunks + 255) / 256;
   if (blocks > 8LL * dev->sms) blocks = 8LL * dev->sms;
@@ -784,7 +818,9 @@ int gqa_attn_decode_append(const void* q, void* k_cache, void* v_cache, const vo
                            unsigned int flags, int causal, int window, float softcap,
                            void* stream) {
   if (flags & GQA_KV_CACHE_F32) return GQA_ATTN_ERR_ARG;  // attention reads bf16 caches
-  if (position < 0 || cache_slots < 0 || (long long)position + q_len > cache_slots)
+  const bool ring = (flags & GQA_KV_RING) != 0;
+  if (position < 0 || cache_slots < 0 ||
+      (long long)position + q_len > (ring ? 0x7fffffffLL : (long long)cache_slots))
     return GQA_ATTN_ERR_ARG;
   Problem pr;
   int rc = validate(batch, q_len, position + q_len, num_q_heads, num_kv_heads, head_dim, causal,
@@ -792,6 +828,7 @@ int gqa_attn_decode_append(const void* q, void* k_cache, void* v_cache, const vo
   if (rc != GQA_ATTN_OK) return rc;
   pr.kv_alloc = cache_slots;
   pr.kv_seq_major = (flags & GQA_KV_CACHE_SEQ_MAJOR) ? 1 : 0;
+  if (ring && (rc = set_ring(&pr, cache_slots)) != GQA_ATTN_OK) return rc;
   rc = check_pointers(pr, q, k_cache, v_cache, o);
   if (rc != GQA_ATTN_OK) return rc;
   const size_t o_bytes = (size_t)batch * num_q_heads * (size_t)q_len * head_dim * 2;
@@ -806,6 +843,22 @@ int gqa_attn_decode_append(const void* q, void* k_cache, void* v_cache, const vo
                           head_dim, position, q_len, flags, nullptr, stream);
   if (rc != GQA_ATTN_OK) return rc;
   return run(pr, q, k_cache, v_cache, o, (cudaStream_t)stream);
+}
+
+int gqa_attn_fwd_ring(const void* q, const void* k_ring, const void* v_ring, void* o, int batch,
+                      int q_len, int kv_len, int ring_slots, int num_q_heads, int num_kv_heads,
+                      int head_dim, unsigned int flags, int causal, int window, float softcap,
+                      void* stream) {
+  if (flags & ~GQA_KV_CACHE_SEQ_MAJOR) return GQA_ATTN_ERR_ARG;
+  Problem pr;
+  int rc = validate(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, causal, window,
+                    softcap, &pr);
+  if (rc != GQA_ATTN_OK) return rc;
+  pr.kv_seq_major = (flags & GQA_KV_CACHE_SEQ_MAJOR) ? 1 : 0;
+  if ((rc = set_ring(&pr, ring_slots)) != GQA_ATTN_OK) return rc;
+  rc = check_pointers(pr, q, k_ring, v_ring, o);
+  if (rc != GQA_ATTN_OK) return rc;
+  return run(pr, q, k_ring, v_ring, o, (cudaStream_t)stream);
 }
 
 const char* gqa_attn_last_error_detail(void) { return g_detail; }

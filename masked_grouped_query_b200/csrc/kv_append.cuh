@@ -27,6 +27,7 @@ struct KvAppendParams {
   const void* new_v;
   int batch, heads, slots, head_dim, position, count;  // count = L
   int cache_seq_major;  // 1: [B][S][H][D], 0: [B][H][S][D]
+  int ring;             // 1: token position + l goes to slot (position + l) % slots
   int new_head_major;   // 1: [B][H][L][D], 0: [B][L][H][D]
 };
 
@@ -43,7 +44,8 @@ __device__ __forceinline__ void kv_append_locate(const KvAppendParams& p, uint32
   const uint32_t outer = p.new_head_major ? p.heads : p.count;
   const uint32_t bb = rest / outer, o = rest % outer;
   const uint32_t l = p.new_head_major ? a : o, h = p.new_head_major ? o : a;
-  const uint32_t slot = (uint32_t)p.position + l;
+  const uint32_t slot = p.ring ? (uint32_t)(((long long)p.position + l) % p.slots)
+                              : (uint32_t)p.position + l;
   const uint64_t dst_row = p.cache_seq_major
                                ? ((uint64_t)bb * p.slots + slot) * p.heads + h
                                : ((uint64_t)bb * p.heads + h) * p.slots + slot;

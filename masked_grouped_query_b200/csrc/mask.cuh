@@ -65,8 +65,10 @@ struct KeyRange {
   int any_lo, any_hi;
 };
 
-__host__ __device__ __forceinline__ KeyRange key_range(const MaskSpec& m, long long r0, int n,
-                                                       int tile) {
+// Tiles here start at key k_base (tile t holds keys k_base + tile*t ..);
+// k_base <= every visible key.  key_range is the k_base = 0 case.
+__host__ __device__ __forceinline__ KeyRange key_range_from(const MaskSpec& m, long long r0, int n,
+                                                            int tile, int k_base) {
   KeyRange kr;
   int qmin, qmax;
   qpos_span(m, r0, n, qmin, qmax);
@@ -78,10 +80,32 @@ __host__ __device__ __forceinline__ KeyRange key_range(const MaskSpec& m, long l
     kr.t_first = 0;
     kr.t_count = 0;
   } else {
-    kr.t_first = kr.any_lo / tile;
-    kr.t_count = kr.any_hi / tile - kr.t_first + 1;
+    kr.t_first = (kr.any_lo - k_base) / tile;
+    kr.t_count = (kr.any_hi - k_base) / tile - kr.t_first + 1;
   }
   return kr;
+}
+
+__host__ __device__ __forceinline__ KeyRange key_range(const MaskSpec& m, long long r0, int n,
+                                                       int tile) {
+  return key_range_from(m, r0, n, tile, 0);
+}
+
+// Ring (circular) K/V storage: key j of a kv_len-key sequence lives in slot
+// j % slots of a ring of `slots` slots (a multiple of `tile`), so the ring
+// holds keys [kv_len - slots, kv_len) once it has wrapped.  Cut the keys
+// into tiles aligned to the ring's slot tiles: with w = kv_len % slots,
+// tile t holds keys k_base + tile*t .. + tile - 1 where
+// k_base = kv_len - slots - (w % tile), and sits in ring slot tile
+// (w / tile + t) % (slots / tile).  Only the first and last of these tiles
+// share a slot tile; each also covers keys that are not in the ring (older
+// than kv_len - slots, or past kv_len), which callers must keep hidden.
+__host__ __device__ __forceinline__ int ring_k_base(int kv_len, int slots, int tile) {
+  const int w = kv_len % slots;
+  return kv_len - slots - (w % tile);
+}
+__host__ __device__ __forceinline__ int ring_phase(int kv_len, int slots, int tile) {
+  return (kv_len % slots) / tile;
 }
 
 }  // namespace gqa

@@ -137,6 +137,15 @@ CACHE_STEPS = {
 }
 
 
+# Single-token grouped-query decode over a 4096-key sliding window kept in a
+# ring of 4096 slots (key j in slot j % 4096) at absolute position 100000.
+RING_STEPS = {
+    "gqa_decode_ring_window": dict(batch=16, q_len=1, kv_len=100000, slots=4096, num_q_heads=32,
+                                   num_kv_heads=8, head_dim=128, causal=True, window=4096,
+                                   softcap=None, seed=6),
+}
+
+
 def make_cache_inputs(batch: int, slots: int, heads: int, head_dim: int, count: int, *,
                       cache_dtype=torch.bfloat16, new_dtype=torch.float32, seed: int = 0,
                       num_q_heads: int | None = None, device="cpu"):

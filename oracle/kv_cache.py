@@ -82,3 +82,37 @@ def kv_update(key_cache: np.ndarray, value_cache: np.ndarray, new_keys: np.ndarr
     kc[:, position:position + length] = convert(new_keys, cache_dtype)
     vc[:, position:position + length] = convert(new_values, cache_dtype)
     return kc, vc, position + length
+
+
+def ring_update(key_ring: np.ndarray, value_ring: np.ndarray, new_keys: np.ndarray,
+                new_values: np.ndarray, position: int):
+    """The update above on ring buffers of S slots: token position + l goes
+    to slot (position + l) % S (a circular window, as in "CSA2 attention on
+    Metal", TensorFold pull request 1709, "What this changes").  L <= S."""
+    cache_dtype = BF16 if key_ring.dtype == np.uint16 else F32
+    b, s, h, d = key_ring.shape
+    nb, length, nh, nd = new_keys.shape
+    if (nb, nh, nd) != (b, h, d) or value_ring.shape != key_ring.shape:
+        raise ValueError("shape mismatch")
+    if position < 0 or length > s:
+        raise ValueError("a block longer than the ring would overwrite itself")
+    kc = key_ring.copy()
+    vc = value_ring.copy()
+    nk = convert(new_keys, cache_dtype)
+    nv = convert(new_values, cache_dtype)
+    for i in range(length):
+        slot = (position + i) % s
+        kc[:, slot] = nk[:, i]
+        vc[:, slot] = nv[:, i]
+    return kc, vc, position + length
+
+
+def ring_sequence(ring: np.ndarray, kv_len: int, fill=0):
+    """Keys (or values) in order from a (B, S, H, D) ring: element j < kv_len
+    of the result, (B, kv_len, H, D), is ring slot j % S for the S most recent
+    keys j >= kv_len - S; older keys are no longer stored and read as `fill`."""
+    b, s, h, d = ring.shape
+    out = np.full((b, kv_len, h, d), fill, dtype=ring.dtype)
+    for j in range(max(0, kv_len - s), kv_len):
+        out[:, j] = ring[:, j % s]
+    return out

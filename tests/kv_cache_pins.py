@@ -12,7 +12,11 @@ it) and raises AssertionError on a mismatch.  They pin it to:
   slots outside [position, position + L) are untouched bit for bit, the new
   block equals the converted new vectors concatenated after the old prefix,
   the returned length is position + L, and bf16 -> fp32 -> bf16 is the
-  identity on every non-NaN bf16 pattern.
+  identity on every non-NaN bf16 pattern;
+* for the ring variant: a hand-worked ring (slot j % S holds key j), and a
+  replay in which a ring and a plain growing sequence receive the same
+  appends in chunks of random sizes -- the ring must read back as the last
+  S keys of the sequence after every step.
 """
 from __future__ import annotations
 
@@ -119,5 +123,41 @@ def pin_update_invariants(kc):
             assert not np.shares_memory(k1, k0)
 
 
+def pin_ring_hand_example(kc):
+    # S = 4 slots, keys 0..5 appended one at a time with value = key index:
+    # slot j % 4 holds key j, so slots 0..3 hold 4, 5, 2, 3 and the stored
+    # keys in order are 2, 3, 4, 5.
+    ring = np.zeros((1, 4, 1, 1), np.float32)
+    for j in range(6):
+        tok = np.full((1, 1, 1, 1), float(j), np.float32)
+        ring, _, n = kc.ring_update(ring, ring, tok, tok, j)
+        assert n == j + 1
+    assert ring[0, :, 0, 0].tolist() == [4.0, 5.0, 2.0, 3.0]
+    seq = kc.ring_sequence(ring, 6, fill=-1.0)
+    assert seq[0, :, 0, 0].tolist() == [-1.0, -1.0, 2.0, 3.0, 4.0, 5.0]
+
+
+def pin_ring_replays_sequence(kc):
+    rng = np.random.default_rng(11)
+    for s_slots in (4, 8):
+        b, h, d = 2, 3, 4
+        ring = np.zeros((b, s_slots, h, d), np.float32)
+        vring = np.zeros_like(ring)
+        seq = np.zeros((b, 0, h, d), np.float32)
+        n = 0
+        while n < 30:
+            length = int(rng.integers(1, s_slots + 1))
+            nk = rng.standard_normal((b, length, h, d)).astype(np.float32)
+            ring, vring, n2 = kc.ring_update(ring, vring, nk, -nk, n)
+            assert n2 == n + length
+            n = n2
+            seq = np.concatenate([seq, nk], axis=1)
+            keep = min(n, s_slots)
+            got = kc.ring_sequence(ring, n)
+            assert np.array_equal(got[:, n - keep:], seq[:, n - keep:]), (s_slots, n)
+            assert np.array_equal(kc.ring_sequence(vring, n)[:, n - keep:], -seq[:, n - keep:])
+
+
 ALL_PINS = [pin_rounding_closed_forms, pin_rounding_matches_torch, pin_round_trip_identity,
-            pin_hand_examples, pin_update_invariants]
+            pin_hand_examples, pin_update_invariants, pin_ring_hand_example,
+            pin_ring_replays_sequence]

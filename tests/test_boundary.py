@@ -82,7 +82,9 @@ def test_append_rejects_bad_arguments_without_a_device(lib):
     assert _append(lib, pos=-1) == -12
     assert _append(lib, pos=8) == -12            # 8 + 1 > 8 slots
     assert _append(lib, pos=5, n=4) == -12
-    assert _append(lib, flags=0x10) == -12       # unknown flag
+    assert _append(lib, flags=0x20) == -12       # unknown flag
+    assert _append(lib, flags=0x10, pos=100) == -7   # ring: any position (then: no device)
+    assert _append(lib, flags=0x10, n=9) == -12      # ring: block larger than the ring
     assert _append(lib, d=60) == -5
     assert _append(lib, h=0) == -3
     assert _append(lib, kc=0) == -1
@@ -107,6 +109,23 @@ def test_append_rejects_bad_arguments_without_a_device(lib):
                                       P(0x110000), P(0x120000), 1, 1, 7, 8, 4, 2, 64, 0,
                                       1, 0, 0.0, None) == -11   # q inside the key cache
     del q, o
+
+
+def _ring(lib, kv_len=5000, slots=4096, q_len=1, window=4096, flags=0, d=64):
+    P = ctypes.c_void_p
+    return lib.gqa_attn_fwd_ring(P(0x10000), P(0x100000), P(0x800000), P(0x2000000), 1, q_len,
+                                 kv_len, slots, 4, 2, d, flags, 1, window, 0.0, None)
+
+
+def test_ring_rejects_bad_arguments_without_a_device(lib):
+    assert _ring(lib, slots=4000) == -12                  # not whole 64-key tiles
+    assert _ring(lib, slots=0) == -12
+    assert _ring(lib, q_len=2) == -12                     # needs window + 1 = 4097 slots
+    assert _ring(lib, window=0) == -12                    # no window: all 5000 keys visible
+    assert _ring(lib, window=0, kv_len=4096) == -7        # they fit: then no device
+    assert _ring(lib, flags=0x2) == -12                   # only the layout flag is accepted
+    assert _ring(lib) == -7
+    assert _ring(lib, flags=0x1) == -7
 
 
 def test_no_device_means_device_error(lib):

@@ -36,9 +36,16 @@ MUTANTS = [
     ("truncation", "out = (upper + round_up.astype(np.uint64)) & 0xFFFF",
      "out = upper & 0xFFFF"),
     ("ties_to_odd", "((upper & 1) == 1)", "((upper & 1) == 0)"),
-    ("length_without_position", "return kc, vc, position + length",
-     "return kc, vc, length"),
+    ("length_without_position",
+     "vc[:, position:position + length] = convert(new_values, cache_dtype)\n    return kc, vc, position + length",
+     "vc[:, position:position + length] = convert(new_values, cache_dtype)\n    return kc, vc, length"),
+    ("ring_length_without_position", "        vc[:, slot] = nv[:, i]\n    return kc, vc, position + length",
+     "        vc[:, slot] = nv[:, i]\n    return kc, vc, length"),
     ("widening_shift", "(b.astype(np.uint32) << 16)", "(b.astype(np.uint32) << 15)"),
+    ("ring_slot_off_by_one", "        slot = (position + i) % s", "        slot = (position + i + 1) % s"),
+    ("ring_read_back_shifted", "        out[:, j] = ring[:, j % s]", "        out[:, j] = ring[:, (j + 1) % s]"),
+    ("ring_keeps_one_too_few", "    for j in range(max(0, kv_len - s), kv_len):",
+     "    for j in range(max(0, kv_len - s + 1), kv_len):"),
     ("no_conversion_for_bf16", "return new.copy() if new.dtype == np.uint16 else "
      "f32_to_bf16_bits(new)", "return new.copy() if new.dtype == np.uint16 else "
      "(new.view(np.uint32) >> 16).astype(np.uint16)"),
