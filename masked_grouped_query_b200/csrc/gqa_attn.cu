@@ -501,6 +501,7 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.ws_ml = ws ? (float*)((char*)ws + pl.off_lse) : nullptr;
   p.tickets = (unsigned int*)tickets;
   p.pair_heads = pl.pair_heads;
+  p.heavy_first = (pr.causal || pr.window > 0) && !pl.split_pairs ? 1 : 0;
   p.causal = pr.causal;
   p.window = pr.window;
   const float rs = 1.0f / std::sqrt((float)pr.d);

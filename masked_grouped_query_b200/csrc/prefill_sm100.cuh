@@ -72,6 +72,7 @@ struct PrefillParams {
                          // key splits 2s and 2s + 1 (units with one row tile)
   int n_items;           // units * pairs_per_unit * splits (/ 2 when split_pairs)
   int pair_heads;        // 1: tiles (2p, 2p+1) are two heads at one position
+  int heavy_first;       // 1: items run in order of decreasing key-tile count (causal / window)
   int causal, window;
   float logit_scale, cap_in, cap_out;
   // Split partials (splits > 1): per (pair, tile, split) O as fp32 [d][128
@@ -176,8 +177,25 @@ __device__ __forceinline__ PfItem prefill_item(const PrefillParams& p, const Mas
   }
   it.split = item % p.splits;
   it.pair_index = item / p.splits;
-  it.unit = it.pair_index / p.pairs_per_unit;
-  const int pair = it.pair_index % p.pairs_per_unit;
+  int pair;
+  if (p.heavy_first) {
+    // Causal / windowed rows see more keys the later their position (up to
+    // the window): walk positions from the last down, all units at each
+    // rank, so the CTAs' last rounds hold the lightest items.
+    const int units = p.n_items / (p.splits * p.pairs_per_unit);
+    const int rank = it.pair_index / units;
+    it.unit = it.pair_index % units;
+    if (p.pair_heads) {
+      const int tiles_per_head = p.q_len / kPfM;
+      const int n_hp = p.pairs_per_unit / tiles_per_head;
+      pair = (rank % n_hp) * tiles_per_head + (tiles_per_head - 1 - rank / n_hp);
+    } else {
+      pair = p.pairs_per_unit - 1 - rank;
+    }
+  } else {
+    it.unit = it.pair_index / p.pairs_per_unit;
+    pair = it.pair_index % p.pairs_per_unit;
+  }
   it.tile[0] = prefill_tile(p, ms, pair, 0);
   it.tile[1] = prefill_tile(p, ms, pair, 1);
   const KeyRange& a = it.tile[0].kr;
@@ -761,9 +779,15 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           const long long blk = (long long)ptile * p.splits;
           float* po = p.ws_o + (blk + psplit) * (long long)p.d_pad * kPfM;
           auto ml_of = [&](int sp) { return p.ws_ml + ((blk + sp) * 2 + h) * 2 * kPfM; };
-          for (int c0 = oc0; c0 < oc1 && have; c0 += 16) {
+          // An empty split writes zeros, so the merge may read every partial.
+          for (int c0 = oc0; c0 < oc1; c0 += 16) {
             float v[16];
-            load_o(c0, v);
+            if (have) {
+              load_o(c0, v);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            }
 #pragma unroll
             for (int e = 0; e < 16; ++e) po[(long long)(c0 + e) * kPfM + r] = v[e];
           }
@@ -778,37 +802,53 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           ticket = __shfl_sync(0xffffffffu, ticket, 0);
           if (ticket == (unsigned)p.splits - 1) {
             __threadfence();
+            // Row max, then row sum, over the splits: eight splits' (m, l)
+            // loads in flight at a time (a split with m = -inf is empty).
             float M = -INFINITY;
-            for (int sp = 0; sp < p.splits; ++sp) M = fmaxf(M, __ldcg(ml_of(sp) + r));
+            for (int sp0 = 0; sp0 < p.splits; sp0 += 8) {
+              float mv[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                mv[i] = sp0 + i < p.splits ? __ldcg(ml_of(sp0 + i) + r) : -INFINITY;
+#pragma unroll
+              for (int i = 0; i < 8; ++i) M = fmaxf(M, mv[i]);
+            }
             float Ls = 0.f;
-            for (int sp = 0; sp < p.splits; ++sp) {
-              const float m = __ldcg(ml_of(sp) + r);
-              Ls += m == -INFINITY ? 0.f : ex2(m - M) * __ldcg(ml_of(sp) + kPfM + r);
+            for (int sp0 = 0; sp0 < p.splits; sp0 += 8) {
+              float mv[8], lv[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const bool in = sp0 + i < p.splits;
+                mv[i] = in ? __ldcg(ml_of(sp0 + i) + r) : -INFINITY;
+                lv[i] = in ? __ldcg(ml_of(sp0 + i) + kPfM + r) : 0.f;
+              }
+#pragma unroll
+              for (int i = 0; i < 8; ++i) Ls += mv[i] == -INFINITY ? 0.f : ex2(mv[i] - M) * lv[i];
             }
             const float inv = Ls > 0.f ? 1.0f / Ls : 0.f;
             store_rows(ti, [&](int col, float (&v)[16]) {
 #pragma unroll
               for (int e = 0; e < 16; ++e) v[e] = 0.f;
-              // Four splits per batch, all their loads in flight together.
+              // Four splits per batch: their m and O loads all in flight
+              // together (every partial was written; past the last split the
+              // loads read split 0 with weight 0).
               for (int sp0 = 0; sp0 < p.splits; sp0 += 4) {
-                float w[4];
+                float mv[4];
                 float x4[4][16];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                  const int sp = sp0 + i;
-                  const float m = sp < p.splits ? __ldcg(ml_of(sp) + r) : -INFINITY;
-                  // empty split (m = -inf): its O was never written
-                  w[i] = m == -INFINITY ? 0.f : ex2(m - M) * inv;
-                  const float* src =
-                      p.ws_o + (blk + (sp < p.splits ? sp : 0)) * (long long)p.d_pad * kPfM + r;
+                  const int sp = sp0 + i < p.splits ? sp0 + i : 0;
+                  mv[i] = sp0 + i < p.splits ? __ldcg(ml_of(sp) + r) : -INFINITY;
+                  const float* src = p.ws_o + (blk + sp) * (long long)p.d_pad * kPfM + r;
 #pragma unroll
-                  for (int e = 0; e < 16; ++e)
-                    x4[i][e] = w[i] != 0.f ? __ldcg(src + (long long)(col + e) * kPfM) : 0.f;
+                  for (int e = 0; e < 16; ++e) x4[i][e] = __ldcg(src + (long long)(col + e) * kPfM);
                 }
 #pragma unroll
-                for (int i = 0; i < 4; ++i)
+                for (int i = 0; i < 4; ++i) {
+                  const float w = mv[i] == -INFINITY ? 0.f : ex2(mv[i] - M) * inv;
 #pragma unroll
-                  for (int e = 0; e < 16; ++e) v[e] += w[i] * x4[i][e];
+                  for (int e = 0; e < 16; ++e) v[e] = fmaf(w, x4[i][e], v[e]);
+                }
               }
             });
             if (lane == 0) atomicExch(tk, 0u);  // ready for the next call
