@@ -446,7 +446,10 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(WORKLOADS))
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=list(WORKLOADS) + list(EXTRA_WORKLOADS),
+                    help="an attention workload, or one of the KV-cache / ring extras "
+                         "(timed alone: one JSON line with its roofline, 1 GPU)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--all", action="store_true", help="also time every other workload")
     ap.add_argument("--no-e2e", action="store_true")
@@ -455,6 +458,13 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if args.workload in EXTRA_WORKLOADS:
+        if args.impl == "reference":
+            if int(os.environ.get("RANK", "0")) == 0:
+                print(json.dumps({"impl": "reference", "unavailable":
+                                  "the oracle arm times the attention workloads only"}))
+            return
+        return run_extra(args)
     w = WORKLOADS[args.workload]
     name, unit, work = metric_of(w)
     pk, pk_src = peaks()
@@ -572,6 +582,43 @@ def main():
             line["other_workloads"] = extra
         print(json.dumps(line))
     ctx.close()
+
+
+EXTRA_WORKLOADS = ("gqa_decode_append", "gqa_decode_ring_window", "kv_append_prompt_block")
+
+
+def run_extra(args):
+    """Time one of the extras alone on GPU 0 and print its line (HBM roofline)."""
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    pk, pk_src = peaks()
+    name = args.workload
+    with ClockSampler(0) as clk:
+        if name in CACHE_STEPS:
+            r = time_cache_step(CACHE_STEPS[name], args.steps, args.warmup, device, _NoDist())
+            metric, launches = "decode step on a KV cache (append + attend) GB/s", 2
+            cfg = {k: v for k, v in vars(CACHE_STEPS[name]).items() if k != "seed"}
+        elif name in RING_STEPS:
+            r = time_ring(RING_STEPS[name], args.steps, args.warmup, device)
+            metric, launches = "masked-GQA attn fwd KV-read GB/s (decode, ring window)", 1
+            cfg = {k: v for k, v in RING_STEPS[name].items() if k != "seed"}
+        else:
+            r = time_kv_append(2, 4096, 4, 128, 4096, args.steps, args.warmup, device)
+            metric, launches = "KV-cache append GB/s (fp32 in, bf16 cache, read + written bytes)", 1
+            cfg = {"batch": 2, "tokens": 4096, "kv_heads": 4, "head_dim": 128, "slots": 4096,
+                   "cache": "(B,S,H,D) bf16", "new": "(B,L,H,D) fp32"}
+    value = r["bytes"] / 1e9 / (r["ms_mean"] * 1e-3)
+    roof = {"bound": "hbm", "achieved": value, "peak": pk["hbm_gbs"], "unit": "GB/s",
+            "frac": value / pk["hbm_gbs"],
+            "peak_source": f"{pk_src} (MEASURED_PEAKS.json)" if pk_src == "measured" else "fallback",
+            "traffic": ncu_traffic(name)}
+    line = {"metric": metric, "value": value, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": r["ms_mean"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": name, **cfg,
+                       "l2": "flushed between timed steps (256 MiB write, then read)"},
+            "roofline": roof, "gpu_launches": launches * args.steps, "clocks": clk.summary()}
+    print(json.dumps(line))
 
 
 class _NoDist:
