@@ -380,17 +380,17 @@ def cpu_sample(w: Workload, budget_s: float = 12.0):
     name, unit, work = metric_of(w)
     per_unit_work = work / units
     # first a single kv-head group to size the sample
+    # Whole groups, cycling through the workload until the time budget is
+    # spent (a workload smaller than the budget is computed several times).
     n_units, elapsed, done = 1, 0.0, 0
     rows_per_unit = g * w.q_len
     while True:
         ids = []
-        for u in range(done, min(units, done + n_units)):
-            b, kvh = divmod(u, w.num_kv_heads)
+        for u in range(done, done + min(n_units, units)):
+            b, kvh = divmod(u % units, w.num_kv_heads)
             for h in range(kvh * g, (kvh + 1) * g):
                 base = (b * w.num_q_heads + h) * w.q_len
                 ids.extend(range(base, base + w.q_len))
-        if not ids:
-            break
         t0 = time.perf_counter()
         oracle.attention_rows(q, k, v, causal=w.causal, window=w.window, softcap=w.softcap,
                               rows=np.asarray(ids, dtype=np.int64), threads=threads)
@@ -398,12 +398,13 @@ def cpu_sample(w: Workload, budget_s: float = 12.0):
         got = len(ids) // rows_per_unit
         done += got
         elapsed += dt
-        if elapsed >= budget_s or done >= units:
+        if elapsed >= budget_s:
             break
-        n_units = max(1, min(units - done, int(got * max(1.0, (budget_s - elapsed) / max(dt, 1e-6)))))
+        n_units = max(1, int(got * max(1.0, (budget_s - elapsed) / max(dt, 1e-6))))
     value = per_unit_work * done / elapsed
-    desc = (f"{done} of {units} (batch, kv head) groups ({done * rows_per_unit} query rows), "
-            f"fp64 oracle, {elapsed:.1f} s")
+    desc = (f"{done} (batch, kv head) groups of {units} in the workload "
+            f"({done * rows_per_unit} query rows; {done / units:.2f} passes), fp64 oracle, "
+            f"{elapsed:.1f} s")
     return value, desc, threads, elapsed
 
 
