@@ -35,6 +35,15 @@ struct DecodeParams {
   int k_base;          // key of tile 0's first column (0, or the ring's key base)
   int ring_tiles;      // ring: slots / 64 (tile t is in slot tile (ring_phase + t) % ring_tiles); 0: none
   int ring_phase;
+  // Fused KV-cache append (app_count > 0): before loading its key tiles, a
+  // CTA writes the new tokens that fall in them into the caches (token l is
+  // key app_pos + l, slot (app_pos + l) % app_slots for a ring).
+  int app_count, app_pos, app_slots, app_ring;
+  int app_new_f32, app_new_head_major, app_cache_seq_major;
+  const void* app_new_k;
+  const void* app_new_v;
+  __nv_bfloat16* app_k_cache;
+  __nv_bfloat16* app_v_cache;
   int rows;            // rows per (b, kvh): group * q_len
   int row_blocks;      // ceil(rows / 64)
   int block_rows;      // min(64, rows): row stride of the partial buffers
@@ -107,6 +116,46 @@ __global__ void __maxnreg__(kT ? 128 : 255)
 
   if (warp == kDecComputeWarps) {
     // ------------------------------------------------------------ loader
+    if (p.app_count > 0 && n_tiles > 0) {
+      // New tokens inside this CTA's key tiles go to the caches first (the
+      // whole warp), then a proxy fence puts the writes ahead of this
+      // warp's TMA loads.  CTAs of other row blocks that load the same
+      // tiles write the same bits.
+      const int b = (int)(unit / p.kv_heads), h = (int)(unit % p.kv_heads);
+      const long long k_lo = (long long)p.k_base + (long long)(kr.t_first + t_begin) * kDecTile;
+      const long long k_hi = k_lo + (long long)n_tiles * kDecTile;  // exclusive
+      const int d8 = p.head_dim / 8;
+      for (int l = 0; l < p.app_count; ++l) {
+        const long long j = (long long)p.app_pos + l;
+        if (j < k_lo || j >= k_hi) continue;
+        const long long slot = p.app_ring ? j % p.app_slots : j;
+        const long long dst_row =
+            p.app_cache_seq_major ? ((long long)b * p.app_slots + slot) * p.kv_heads + h
+                                  : ((long long)b * p.kv_heads + h) * p.app_slots + slot;
+        const long long src_row = p.app_new_head_major
+                                      ? ((long long)b * p.kv_heads + h) * p.app_count + l
+                                      : ((long long)b * p.app_count + l) * p.kv_heads + h;
+        for (int c = lane; c < 2 * d8; c += 32) {  // 8 elements per step, keys then values
+          const int kv = c >= d8, c8 = kv ? c - d8 : c;
+          const long long src = src_row * p.head_dim + 8 * c8;
+          uint4 w;
+          if (p.app_new_f32) {
+            const float4* s4 =
+                reinterpret_cast<const float4*>(static_cast<const float*>(kv ? p.app_new_v : p.app_new_k) + src);
+            const float4 x0 = s4[0], x1 = s4[1];
+            w = make_uint4(pack_bf16(x0.x, x0.y), pack_bf16(x0.z, x0.w), pack_bf16(x1.x, x1.y),
+                           pack_bf16(x1.z, x1.w));
+          } else {
+            w = *reinterpret_cast<const uint4*>(
+                static_cast<const __nv_bfloat16*>(kv ? p.app_new_v : p.app_new_k) + src);
+          }
+          *reinterpret_cast<uint4*>((kv ? p.app_v_cache : p.app_k_cache) +
+                                    dst_row * p.head_dim + 8 * c8) = w;
+        }
+      }
+      fence_proxy_async_global();
+      __syncwarp();
+    }
     if (lane == 0 && n_tiles > 0) {
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);

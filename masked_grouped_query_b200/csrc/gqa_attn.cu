@@ -84,6 +84,10 @@ struct Problem {
   long long kv_alloc;  // key slots allocated per (batch, kv head): kv_len, or a cache's slots
   int kv_seq_major;    // 0: k/v [batch][hkv][kv_alloc][d]; 1: [batch][kv_alloc][hkv][d]
   int ring;            // ring of `ring` slots (key j in slot j % ring); 0: keys in order
+  // KV-cache append fused into the split-KV decode kernel (app_count > 0).
+  int app_count = 0, app_pos = 0, app_new_f32 = 0, app_new_head_major = 0;
+  const void* app_new_k = nullptr;
+  const void* app_new_v = nullptr;
 };
 
 int validate(int batch, int q_len, int kv_len, int hq, int hkv, int d, int causal, int window,
@@ -416,6 +420,17 @@ int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.k_base = pr.ring ? ring_k_base(pr.kv_len, pr.ring, kDecTile) : 0;
   p.ring_tiles = pr.ring ? pr.ring / kDecTile : 0;
   p.ring_phase = pr.ring ? ring_phase(pr.kv_len, pr.ring, kDecTile) : 0;
+  p.app_count = pr.app_count;
+  p.app_pos = pr.app_pos;
+  p.app_slots = (int)pr.kv_alloc;
+  p.app_ring = pr.ring ? 1 : 0;
+  p.app_new_f32 = pr.app_new_f32;
+  p.app_new_head_major = pr.app_new_head_major;
+  p.app_cache_seq_major = pr.kv_seq_major;
+  p.app_new_k = pr.app_new_k;
+  p.app_new_v = pr.app_new_v;
+  p.app_k_cache = (__nv_bfloat16*)k;
+  p.app_v_cache = (__nv_bfloat16*)v;
   p.head_dim = pr.d;
   p.rows = (int)pr.rows;
   p.row_blocks = pl.row_blocks;
@@ -750,9 +765,13 @@ int gqa_attn_selftest_bounded_wait(int limit_us, void* stream) {
 
 int gqa_attn_version(void) { return 200; }
 
-int gqa_attn_kv_append(void* k_cache, void* v_cache, const void* new_k, const void* new_v,
-                       int batch, int cache_slots, int num_kv_heads, int head_dim, int position,
-                       int count, unsigned int flags, int* new_length, void* stream) {
+// Argument checks of a KV-cache append (nothing launched).  *n_out gets the
+// number of new elements per tensor; GQA_ATTN_OK with *n_out == 0 means
+// there is nothing to write.
+static int append_checks(void* k_cache, void* v_cache, const void* new_k, const void* new_v,
+                         int batch, int cache_slots, int num_kv_heads, int head_dim,
+                         int position, int count, unsigned int flags, long long* n_out) {
+  *n_out = 0;
   if (flags & ~(GQA_KV_CACHE_SEQ_MAJOR | GQA_KV_CACHE_F32 | GQA_KV_NEW_BF16 |
                 GQA_KV_NEW_HEAD_MAJOR | GQA_KV_RING))
     return GQA_ATTN_ERR_ARG;
@@ -764,7 +783,6 @@ int gqa_attn_kv_append(void* k_cache, void* v_cache, const void* new_k, const vo
       (ring && count > cache_slots))
     return GQA_ATTN_ERR_ARG;
   const long long n = (long long)batch * num_kv_heads * count * head_dim;
-  if (new_length) *new_length = position + count;
   if (n == 0) return GQA_ATTN_OK;
   if (2 * n / 8 + 4LL * 8 * 1024 * 256 >= (1LL << 32)) {  // chunk indices are 32-bit
     snprintf(g_detail, sizeof g_detail, "kv_append: %lld new elements exceed the 32-bit index",
@@ -783,8 +801,22 @@ int gqa_attn_kv_append(void* k_cache, void* v_cache, const void* new_k, const vo
       overlaps(new_v, new_bytes, k_cache, cache_bytes) ||
       overlaps(new_v, new_bytes, v_cache, cache_bytes))
     return GQA_ATTN_ERR_ALIAS;
+  *n_out = n;
+  return GQA_ATTN_OK;
+}
+
+int gqa_attn_kv_append(void* k_cache, void* v_cache, const void* new_k, const void* new_v,
+                       int batch, int cache_slots, int num_kv_heads, int head_dim, int position,
+                       int count, unsigned int flags, int* new_length, void* stream) {
+  long long n = 0;
+  int rc = append_checks(k_cache, v_cache, new_k, new_v, batch, cache_slots, num_kv_heads,
+                         head_dim, position, count, flags, &n);
+  if (rc != GQA_ATTN_OK) return rc;
+  if (new_length) *new_length = position + count;
+  if (n == 0) return GQA_ATTN_OK;
+  const bool ring = (flags & GQA_KV_RING) != 0;
   DeviceInfo* dev = nullptr;
-  int rc = device_info(&dev);
+  rc = device_info(&dev);
   if (rc != GQA_ATTN_OK) return rc;
   KvAppendParams p;
   p.k_cache = k_cache;
@@ -840,6 +872,24 @@ int gqa_attn_decode_append(const void* q, void* k_cache, void* v_cache, const vo
   if (overlaps(o, o_bytes, new_k, new_bytes) || overlaps(o, o_bytes, new_v, new_bytes) ||
       overlaps(q, q_bytes, k_cache, cache_bytes) || overlaps(q, q_bytes, v_cache, cache_bytes))
     return GQA_ATTN_ERR_ALIAS;
+  long long n_new = 0;
+  rc = append_checks(k_cache, v_cache, new_k, new_v, batch, cache_slots, num_kv_heads, head_dim,
+                     position, q_len, flags, &n_new);
+  if (rc != GQA_ATTN_OK || n_new == 0) return rc;
+  DeviceInfo* dev = nullptr;
+  if ((rc = device_info(&dev)) != GQA_ATTN_OK) return rc;
+  Plan pl;
+  if ((rc = make_plan(pr, *dev, &pl)) != GQA_ATTN_OK) return rc;
+  if (pl.path == kPathDecode) {
+    // One launch: the decode kernel writes the new tokens itself.
+    pr.app_count = q_len;
+    pr.app_pos = position;
+    pr.app_new_f32 = (flags & GQA_KV_NEW_BF16) ? 0 : 1;
+    pr.app_new_head_major = (flags & GQA_KV_NEW_HEAD_MAJOR) ? 1 : 0;
+    pr.app_new_k = new_k;
+    pr.app_new_v = new_v;
+    return run(pr, q, k_cache, v_cache, o, (cudaStream_t)stream);
+  }
   rc = gqa_attn_kv_append(k_cache, v_cache, new_k, new_v, batch, cache_slots, num_kv_heads,
                           head_dim, position, q_len, flags, nullptr, stream);
   if (rc != GQA_ATTN_OK) return rc;
