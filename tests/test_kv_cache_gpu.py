@@ -136,6 +136,8 @@ DECODE_STEPS = [
     (1, 300, 0, 200, 4, 4, 64, True, 64, 20.0, False, torch.float32),      # from empty
     (3, 520, 77, 3, 12, 4, 96, False, None, None, False, torch.bfloat16),
     (2, 4100, 4000, 2, 16, 16, 72, True, 1000, None, True, torch.float32),
+    (2, 600, 500, 20, 8, 2, 256, True, None, None, True, torch.float32),   # 2 row blocks write
+    (1, 1100, 1000, 30, 4, 1, 256, True, 700, 25.0, False, torch.bfloat16),  # tokens span 2 tiles
 ]
 
 
@@ -190,3 +192,15 @@ def test_decode_append_bench_workload_sampled():
     want = oracle.attention_rows(x["q"].cpu(), k_used, v_used, causal=st.causal,
                                  window=st.window, softcap=st.softcap, rows=rows)
     assert_close(out.reshape(-1, st.head_dim)[torch.as_tensor(rows)], want, st.name)
+
+
+def test_fused_append_with_one_tile_per_split():
+    """Every 64-key tile its own CTA: new tokens that straddle a tile edge
+    are written by two CTAs, each before its own loads (decode kernel,
+    head_dim 256, two row blocks)."""
+    step = (1, 1100, 1000, 30, 4, 1, 256, True, None, None, True, torch.float32)
+    mgq.set_override("tiles_per_split", 1)
+    try:
+        test_decode_append_matches_oracle(step)
+    finally:
+        mgq.set_override("tiles_per_split", 0)
