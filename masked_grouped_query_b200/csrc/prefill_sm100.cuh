@@ -95,8 +95,8 @@ struct PrefillCfg {
   // Row values swapped between the two column halves: [half][row] fp32.
   static constexpr int kXchgBytes = 2 * 128 * 4;
   static constexpr int kBarOffset = kQBytes + kRingBytes + kStageBytes + kXchgBytes;
-  // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain
-  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 1;
+  // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, drain
+  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 1 + 1;
   static constexpr int kSmemBytes = 1024 + kBarOffset + kNumBars * 8 + 16;
 };
 
@@ -261,8 +261,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* kv_empty = kv_full + C::kSlots;
   uint64_t* s_full = kv_empty + C::kSlots;
   uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 2;
-  uint64_t* drain = o_done + 2;
+  uint64_t* o_done = p_full + 2;  // every MMA of an item has finished
+  uint64_t* drain = o_done + 1;
   uint32_t* tmem_slot = (uint32_t*)(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -278,8 +278,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 256);
-      mbar_init(&o_done[t], 1);
     }
+    mbar_init(o_done, 1);
     mbar_init(drain, 1);
     fence_barrier_init();
   }
@@ -428,8 +428,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
           }
           if (!ok) break;
-          mma_commit(&o_done[0]);
-          mma_commit(&o_done[1]);
+          mma_commit(o_done);
           ubase += paired_pos(it, 0, it.j_count, 0);
           continue;
         }
@@ -471,8 +470,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (j + 1 < it.j_count) release(2 * (j + 1));
         }
         if (!ok) break;
-        mma_commit(&o_done[0]);
-        mma_commit(&o_done[1]);
+        mma_commit(o_done);
         ubase += 2 * it.j_count;
       }
       // Drain: every MMA finished before TMEM can be released.
@@ -702,7 +700,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // covers both tiles: every MMA of the item has finished.
       bool eok = true;
       if (it.busy) {
-        eok = __all_sync(0xffffffffu, mbar_wait(&o_done[0], n_done & 1, kStatusTimeoutEpilogue));
+        eok = __all_sync(0xffffffffu, mbar_wait(o_done, n_done & 1, kStatusTimeoutEpilogue));
         ++n_done;
       }
       // Row sums: the two halves add the same two values in the same order.

@@ -1,0 +1,42 @@
+"""The attention call inside a CUDA graph (GPU).
+
+After one call on a stream (which sizes that stream's split workspace), a
+call enqueues only kernels -- no allocation, no host synchronisation -- so a
+serving loop can capture it once and replay it: the tensor maps and plan are
+baked in at capture, and replays read whatever the captured buffers hold.
+"""
+import pytest
+import torch
+
+import masked_grouped_query_b200 as mgq
+from masked_grouped_query_b200.inputs import Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("w", [
+    Workload("decode", 4, 1, 3000, 32, 8, 128, True, None, None, 31),         # split-KV decode
+    Workload("prefill", 1, 300, 900, 8, 2, 128, True, 256, 30.0, 32),         # tcgen05, key splits
+])
+def test_captured_call_replays_like_a_direct_call(w):
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    out = torch.empty_like(q)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        mgq.attention(q, k, v, causal=w.causal, window=w.window, softcap=w.softcap, out=out)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        mgq.attention(q, k, v, causal=w.causal, window=w.window, softcap=w.softcap, out=out)
+    for seed in (1, 2):
+        q2, k2, v2 = make_inputs(w, seed=100 + seed)
+        q.copy_(q2)
+        k.copy_(k2)
+        v.copy_(v2)
+        g.replay()
+        torch.cuda.synchronize()
+        want = mgq.attention(q, k, v, causal=w.causal, window=w.window, softcap=w.softcap)
+        torch.cuda.synchronize()
+        assert torch.equal(out, want)
+    assert mgq.status() & 0x1f == 0
