@@ -36,7 +36,7 @@ struct DeviceInfo {
   int sms = 0, major = 0, minor = 0;
   int smem_optin = 0;
   bool decode_attr[8] = {false, false, false, false, false, false, false, false};
-  bool prefill_attr[4] = {false, false, false, false};
+  bool prefill_attr[6] = {false, false, false, false, false, false};
 };
 
 std::mutex g_mu;
@@ -472,16 +472,18 @@ int launch_decode(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void
   }
 }
 
-template <int DCH, bool kCap>
+template <int DCH, int kCapDeg>
 int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
                      const void* k, const void* v, void* o, void* ws, void* tickets,
                      cudaStream_t stream) {
   using C = PrefillCfg<DCH>;
-  if (!dev.prefill_attr[(DCH - 1) + (kCap ? 2 : 0)]) {
+  constexpr bool kCap = kCapDeg != 0;
+  constexpr int attr = (DCH - 1) + (kCapDeg == 5 ? 2 : kCapDeg == 7 ? 4 : 0);
+  if (!dev.prefill_attr[attr]) {
     // The register split inside the kernel must fit what the block is
     // launched with, or setmaxnreg.inc could never be granted.
     cudaFuncAttributes fa;
-    const cudaError_t ea = cudaFuncGetAttributes(&fa, prefill_sm100_kernel<DCH, kCap>);
+    const cudaError_t ea = cudaFuncGetAttributes(&fa, prefill_sm100_kernel<DCH, kCapDeg>);
     if (ea != cudaSuccess) return cuda_fail("cudaFuncGetAttributes(prefill)", ea, GQA_ATTN_ERR_LAUNCH);
     if ((long long)fa.numRegs * kPfThreads < kRegSplitTotal) {
       snprintf(g_detail, sizeof g_detail, "prefill kernel built with %d registers/thread: "
@@ -489,9 +491,9 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
       return GQA_ATTN_ERR_LAUNCH;
     }
     const cudaError_t e = cudaFuncSetAttribute(
-        prefill_sm100_kernel<DCH, kCap>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        prefill_sm100_kernel<DCH, kCapDeg>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(prefill)", e, GQA_ATTN_ERR_LAUNCH);
-    dev.prefill_attr[(DCH - 1) + (kCap ? 2 : 0)] = true;
+    dev.prefill_attr[attr] = true;
   }
   CUtensorMap tq, tk, tv, to;
   if (encode_map(&tq, q, pr.d, pr.rows, pr.units, kPfM) != GQA_ATTN_OK ||
@@ -525,7 +527,7 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.cap_out = kCap ? pr.softcap * kLog2e : 0.f;
   // Persistent: at most one CTA per SM, each walking items with stride grid.
   const int grid = (int)(pl.ctas < dev.sms ? pl.ctas : dev.sms);
-  prefill_sm100_kernel<DCH, kCap><<<dim3((unsigned)grid), kPfThreads, C::kSmemBytes, stream>>>(
+  prefill_sm100_kernel<DCH, kCapDeg><<<dim3((unsigned)grid), kPfThreads, C::kSmemBytes, stream>>>(
       tq, tk, tv, to, p);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? GQA_ATTN_OK : cuda_fail("launch(prefill)", e, GQA_ATTN_ERR_LAUNCH);
@@ -534,11 +536,15 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
 int launch_prefill(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
                    const void* k, const void* v, void* o, void* ws, void* tickets,
                    cudaStream_t stream) {
+  // Softcaps up to kTanh5MaxCap take the degree-5 tanh polynomial.
+  if (pr.softcap > 0.f && pr.softcap <= kTanh5MaxCap)
+    return pl.dch == 1 ? launch_prefill_d<1, 5>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
+                       : launch_prefill_d<2, 5>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
   if (pr.softcap > 0.f)
-    return pl.dch == 1 ? launch_prefill_d<1, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
-                       : launch_prefill_d<2, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
-  return pl.dch == 1 ? launch_prefill_d<1, false>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
-                     : launch_prefill_d<2, false>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+    return pl.dch == 1 ? launch_prefill_d<1, 7>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
+                       : launch_prefill_d<2, 7>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+  return pl.dch == 1 ? launch_prefill_d<1, 0>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
+                     : launch_prefill_d<2, 0>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
 }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {

@@ -241,13 +241,17 @@ __device__ __forceinline__ int paired_pos(const PfItem& it, int t, int j, int kv
   return 2 * j + 2 * min(j, it.kc[1]) + 2 * t + kv;
 }
 
-template <int DCH, bool kCap>
+// kCapDeg: 0 = no softcap; 5 or 7 = softcap, with the odd polynomial of that
+// degree for tanh of small arguments (5 where the cap is small enough for its
+// error, see kTanh5C*).
+template <int DCH, int kCapDeg>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v,
                          const __grid_constant__ CUtensorMap tm_o, const PrefillParams p) {
   using C = PrefillCfg<DCH>;
+  constexpr bool kCap = kCapDeg != 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* sq = smem;                   // Q tiles A, B
@@ -661,17 +665,28 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             // zeroed explicitly.
             auto hidden = [&](int col) { return x[col] == -INFINITY; };
             if (small_y) {
-              // tanh_poly_small's coefficients with cap_in^(2k+1) * cap_out
-              // folded in: cap_out * tanh(x * cap_in) = x * Q(x^2).
+              // The odd tanh polynomial with cap_in^(2k+1) * cap_out folded
+              // in: cap_out * tanh(x * cap_in) = x * Q(x^2).
               const float ci2 = p.cap_in * p.cap_in, cc = p.cap_out * p.cap_in;
-              const float q0 = cc * kTanhC1, q1 = cc * ci2 * kTanhC3;
-              const float q2c = cc * ci2 * ci2 * kTanhC5, q3 = cc * ci2 * ci2 * ci2 * kTanhC7;
-              auto logit = [&](float v) {
-                const float v2 = v * v;
-                return fmaf(v, fmaf(fmaf(fmaf(q3, v2, q2c), v2, q1), v2, q0), -base);
-              };
-              if (need_mask) emit(logit, hidden);
-              else emit(logit, none);
+              if constexpr (kCapDeg == 5) {
+                const float q0 = cc * kTanh5C1, q1 = cc * ci2 * kTanh5C3;
+                const float q2c = cc * ci2 * ci2 * kTanh5C5;
+                auto logit = [&](float v) {
+                  const float v2 = v * v;
+                  return fmaf(v, fmaf(fmaf(q2c, v2, q1), v2, q0), -base);
+                };
+                if (need_mask) emit(logit, hidden);
+                else emit(logit, none);
+              } else {
+                const float q0 = cc * kTanhC1, q1 = cc * ci2 * kTanhC3;
+                const float q2c = cc * ci2 * ci2 * kTanhC5, q3 = cc * ci2 * ci2 * ci2 * kTanhC7;
+                auto logit = [&](float v) {
+                  const float v2 = v * v;
+                  return fmaf(v, fmaf(fmaf(fmaf(q3, v2, q2c), v2, q1), v2, q0), -base);
+                };
+                if (need_mask) emit(logit, hidden);
+                else emit(logit, none);
+              }
             } else {
               const float co = p.cap_out, ci = p.cap_in;
               auto logit = [&](float v) { return fmaf(co, tanh_fast(v * ci), -base); };

@@ -123,6 +123,16 @@ def test_softcap_saturating_inputs():
         check_workload(w2, q_scale=20.0)
 
 
+def test_softcap_polynomial_degrees():
+    # Caps up to 256 take the degree-5 tanh polynomial in the tcgen05
+    # kernel, larger ones the degree-7 one; both against the oracle, with
+    # q scaled so the logits span tens of units.
+    for cap, seed in ((200.0, 41), (300.0, 42), (1000.0, 43)):
+        w = Workload("capdeg", 1, 200, 300, 8, 2, 128, True, None, cap, seed=seed)
+        assert mgq.describe(1, 200, 300, 8, 2, 128, True, None, cap)["path"] == "prefill"
+        check_workload(w, q_scale=8.0)
+
+
 def test_constant_v_returns_v():
     w = Workload("c", 2, 4, 700, 16, 4, 128, True, 300, 30.0, 8)
     q, k, _ = make_inputs(w)
