@@ -36,7 +36,7 @@ struct DeviceInfo {
   int sms = 0, major = 0, minor = 0;
   int smem_optin = 0;
   bool decode_attr[8] = {false, false, false, false, false, false, false, false};
-  bool prefill_attr[6] = {false, false, false, false, false, false};
+  bool prefill_attr[12] = {};  // per (DCH, softcap degree, split) instantiation
 };
 
 std::mutex g_mu;
@@ -235,13 +235,14 @@ int plan_prefill(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
     pl->splits = (int)(2 * half);
     pl->pairs_per_unit = 1;
     pl->ctas = pr.units * half;
+    // One partial per item (its two splits are combined in the kernel):
+    // O as fp32, and (m, l) per column half of the softmax, per row.
     const size_t tiles = (size_t)pr.units;
-    pl->ws_bytes = align256(tiles * pl->splits * (size_t)pl->d_pad * kPfM * 4);
+    pl->ws_bytes = align256(tiles * half * (size_t)pl->d_pad * kPfM * 4);
     pl->off_lse = pl->ws_bytes;
-    // (m, l) per split, per column half of the softmax, per row
-    pl->ws_bytes += align256(tiles * pl->splits * 2 * 2 * kPfM * 4);
-    // one ticket per (tile, lane quarter, column half)
-    pl->ticket_bytes = align256(tiles * 8 * sizeof(unsigned int));
+    pl->ws_bytes += align256(tiles * half * 2 * 2 * kPfM * 4);
+    // one ticket per (tile, column half)
+    pl->ticket_bytes = align256(tiles * 2 * sizeof(unsigned int));
     return GQA_ATTN_OK;
   }
   const long long pairs = pl->ctas;
@@ -256,7 +257,7 @@ int plan_prefill(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
     pl->ws_bytes = align256((size_t)pairs * 2 * pl->splits * (size_t)pl->d_pad * kPfM * 4);
     pl->off_lse = pl->ws_bytes;
     pl->ws_bytes += align256((size_t)pairs * 2 * pl->splits * 2 * 2 * kPfM * 4);
-    pl->ticket_bytes = align256((size_t)pairs * 2 * 8 * sizeof(unsigned int));
+    pl->ticket_bytes = align256((size_t)pairs * 2 * 2 * sizeof(unsigned int));
   }
   return GQA_ATTN_OK;
 }
@@ -472,18 +473,18 @@ int launch_decode(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void
   }
 }
 
-template <int DCH, int kCapDeg>
-int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
+template <int DCH, int kCapDeg, bool kSplit>
+int launch_prefill_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
                      const void* k, const void* v, void* o, void* ws, void* tickets,
                      cudaStream_t stream) {
   using C = PrefillCfg<DCH>;
   constexpr bool kCap = kCapDeg != 0;
-  constexpr int attr = (DCH - 1) + (kCapDeg == 5 ? 2 : kCapDeg == 7 ? 4 : 0);
+  constexpr int attr = (DCH - 1) + (kCapDeg == 5 ? 2 : kCapDeg == 7 ? 4 : 0) + (kSplit ? 6 : 0);
   if (!dev.prefill_attr[attr]) {
     // The register split inside the kernel must fit what the block is
     // launched with, or setmaxnreg.inc could never be granted.
     cudaFuncAttributes fa;
-    const cudaError_t ea = cudaFuncGetAttributes(&fa, prefill_sm100_kernel<DCH, kCapDeg>);
+    const cudaError_t ea = cudaFuncGetAttributes(&fa, prefill_sm100_kernel<DCH, kCapDeg, kSplit>);
     if (ea != cudaSuccess) return cuda_fail("cudaFuncGetAttributes(prefill)", ea, GQA_ATTN_ERR_LAUNCH);
     if ((long long)fa.numRegs * kPfThreads < kRegSplitTotal) {
       snprintf(g_detail, sizeof g_detail, "prefill kernel built with %d registers/thread: "
@@ -491,7 +492,7 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
       return GQA_ATTN_ERR_LAUNCH;
     }
     const cudaError_t e = cudaFuncSetAttribute(
-        prefill_sm100_kernel<DCH, kCapDeg>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        prefill_sm100_kernel<DCH, kCapDeg, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(prefill)", e, GQA_ATTN_ERR_LAUNCH);
     dev.prefill_attr[attr] = true;
   }
@@ -527,10 +528,19 @@ int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.cap_out = kCap ? pr.softcap * kLog2e : 0.f;
   // Persistent: at most one CTA per SM, each walking items with stride grid.
   const int grid = (int)(pl.ctas < dev.sms ? pl.ctas : dev.sms);
-  prefill_sm100_kernel<DCH, kCapDeg><<<dim3((unsigned)grid), kPfThreads, C::kSmemBytes, stream>>>(
+  prefill_sm100_kernel<DCH, kCapDeg, kSplit><<<dim3((unsigned)grid), kPfThreads, C::kSmemBytes, stream>>>(
       tq, tk, tv, to, p);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? GQA_ATTN_OK : cuda_fail("launch(prefill)", e, GQA_ATTN_ERR_LAUNCH);
+}
+
+template <int DCH, int kCapDeg>
+int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
+                     const void* k, const void* v, void* o, void* ws, void* tickets,
+                     cudaStream_t stream) {
+  return pl.splits > 1
+             ? launch_prefill_k<DCH, kCapDeg, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
+             : launch_prefill_k<DCH, kCapDeg, false>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
 }
 
 int launch_prefill(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,

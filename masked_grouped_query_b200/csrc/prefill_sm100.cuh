@@ -17,12 +17,14 @@
 // Roles (12 warps, three warpgroups):
 //   warp 0      TMA loader: Q tiles, then K_j, V_j (128 keys x head_dim,
 //               128-byte swizzle) into a ring of shared-memory slots guarded
-//               by mbarriers;
+//               by mbarriers (for paired items, below, K only: warp 2
+//               streams V through its own half of the ring);
 //   warp 1      TMEM allocator and single-thread tcgen05.mma issuer:
 //               S_t = Q_t K_j^T (M=128, N=128, fp32 in TMEM) and
 //               O_t += P_t V_j (A = P from TMEM, B = V from shared memory,
 //               N = head_dim rounded up to 16);
-//   warps 2-3   idle (they complete warpgroup 0 for the register split);
+//   warps 2-3   idle but for warp 2's V stream of paired items (they
+//               complete warpgroup 0 for the register split);
 //   warps 4-11  softmax + epilogue: warps 4-7 take key columns [0, 64) of
 //               each S tile, warps 8-11 columns [64, 128).  A thread owns
 //               half of one row: it reads that half from TMEM, applies
@@ -75,8 +77,9 @@ struct PrefillParams {
   int heavy_first;       // 1: items run in order of decreasing key-tile count (causal / window)
   int causal, window;
   float logit_scale, cap_in, cap_out;
-  // Split partials (splits > 1): per (pair, tile, split) O as fp32 [d][128
-  // rows] (column-major, so a warp's accesses coalesce) and (m, l) per row;
+  // Split partials (splits > 1): per (pair, tile, split) O as fp32
+  // [d / 4][128 rows][4] (a thread moves four columns of its row as one
+  // 16-byte access and a warp's accesses coalesce) and (m, l) per row;
   // tickets per (pair, tile, warp) count the splits that have finished.
   float* ws_o;
   float* ws_ml;
@@ -95,8 +98,9 @@ struct PrefillCfg {
   // Row values swapped between the two column halves: [half][row] fp32.
   static constexpr int kXchgBytes = 2 * 128 * 4;
   static constexpr int kBarOffset = kQBytes + kRingBytes + kStageBytes + kXchgBytes;
-  // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, drain
-  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 1 + 1;
+  // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, drain,
+  // part_done[2], flag_ready[2]
+  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 1 + 1 + 2 + 2;
   static constexpr int kSmemBytes = 1024 + kBarOffset + kNumBars * 8 + 16;
 };
 
@@ -147,10 +151,11 @@ struct PfItem {
   bool busy;
 };
 
+template <bool kSplit>
 __device__ __forceinline__ PfItem prefill_item(const PrefillParams& p, const MaskSpec& ms,
                                                int item) {
   PfItem it;
-  it.paired = p.split_pairs != 0;
+  it.paired = kSplit && p.split_pairs != 0;
   if (it.paired) {
     const int half = p.splits / 2;
     it.split = 2 * (item % half);
@@ -210,7 +215,7 @@ __device__ __forceinline__ PfItem prefill_item(const PrefillParams& p, const Mas
     it.j_first = min(fa, fb);
     it.j_count = max(la, lb) - it.j_first + 1;
   }
-  if (p.splits > 1) {  // this item's share of the key tiles
+  if (kSplit && p.splits > 1) {  // this item's share of the key tiles
     const int per = (it.j_count + p.splits - 1) / p.splits;
     const int js = min(it.j_count, it.split * per), je = min(it.j_count, js + per);
     it.j_first += js;
@@ -234,17 +239,11 @@ __device__ __forceinline__ int key_tile(const PfItem& it, int t, int j) {
   return (t == 0 ? it.kt0[0] : it.kt0[1]) + j;
 }
 
-// Ring position (relative to the item's first load) of K (kv = 0) or V
-// (kv = 1) for tile t at iteration j when paired: each iteration loads K, V
-// of tile 0, then K, V of tile 1 while tile 1 is active.
-__device__ __forceinline__ int paired_pos(const PfItem& it, int t, int j, int kv) {
-  return 2 * j + 2 * min(j, it.kc[1]) + 2 * t + kv;
-}
-
 // kCapDeg: 0 = no softcap; 5 or 7 = softcap, with the odd polynomial of that
 // degree for tanh of small arguments (5 where the cap is small enough for its
-// error, see kTanh5C*).
-template <int DCH, int kCapDeg>
+// error, see kTanh5C*).  kSplit: items cover key-range splits (splits > 1),
+// whose partials are merged; without it the split code is not compiled in.
+template <int DCH, int kCapDeg, bool kSplit>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -267,7 +266,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* p_full = s_full + 2;
   uint64_t* o_done = p_full + 2;  // every MMA of an item has finished
   uint64_t* drain = o_done + 1;
-  uint32_t* tmem_slot = (uint32_t*)(drain + 1);
+  // Key splits: the four warps of a column half have written their partials
+  // (part_done[h]), and the ticket's answer is in merge_flag[h] (flag_ready[h]).
+  uint64_t* part_done = drain + 1;
+  uint64_t* flag_ready = part_done + 2;
+  uint32_t* tmem_slot = (uint32_t*)(flag_ready + 2);
+  int* merge_flag = (int*)(tmem_slot + 1);  // [2]: 1 merge, 0 not the last, -1 wait gave up
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const MaskSpec ms{p.q_len, p.kv_len, p.causal, p.window};
@@ -285,6 +289,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&part_done[t], 128);
+      mbar_init(&flag_ready[t], 1);
+    }
     fence_barrier_init();
   }
   if (warp == 1) {
@@ -301,57 +309,87 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
   }
-  if (warp == 0) {
-    // ------------------------------------------------------------ loader
+  if (warp == 0 || (kSplit && warp == 2 && p.split_pairs)) {
+    // ------------------------------------------------------------ loaders
+    // Paired items (split_pairs): K and V have sub-rings of kSlots / 2 slots
+    // each, streamed by two threads (warp 0: Q and K, warp 2: V), so a K
+    // tile never queues behind a V slot that waits for the softmax.
+    // Otherwise warp 0 streams Q and K_j, V_j through the whole ring.
     if (lane == 0) {
-      tma_prefetch_map(&tm_q);
+      constexpr int kHalf = C::kSlots / 2;
+      const bool v_stream = kSplit && warp == 2;
+      if (!v_stream) tma_prefetch_map(&tm_q);
       tma_prefetch_map(&tm_k);
       tma_prefetch_map(&tm_v);
-      int u = 0;       // K/V tiles issued (ring position)
+      int u = 0;       // K/V tiles issued (ring position, or stream position when paired)
       int nq = 0;      // busy items whose Q was issued
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-        const PfItem it = prefill_item(p, ms, item);
+        const PfItem it = prefill_item<kSplit>(p, ms, item);
         if (!it.busy) continue;
-        // The Q buffer is free once every S of the previous busy item is done.
-        if (nq > 0 && !(ok = mbar_wait(q_empty, (nq - 1) & 1, kStatusTimeoutProducer))) break;
-        // Paired items share tile 0's Q.
-        const int qtiles = it.paired ? 1 : 2;
-        int ntiles = 0;
-        for (int t = 0; t < qtiles; ++t) ntiles += it.tile[t].nrows > 0 ? 1 : 0;
-        mbar_arrive_expect_tx(q_full, ntiles * C::kTileBytes);
-        for (int t = 0; t < qtiles; ++t)
-          if (it.tile[t].nrows > 0)
-            for (int c = 0; c < DCH; ++c)
-              tma_load_3d(sq + t * C::kTileBytes + c * C::kBoxBytes, &tm_q, q_full, c * 64,
-                          it.tile[t].row0, it.unit);
-        ++nq;
-        for (int j = 0; j < it.j_count && ok; ++j) {
-          // One K/V stream per iteration, or one per active tile when paired.
-          const int streams = it.paired ? (tile_active(it, 1, j) ? 2 : 1) : 1;
-          for (int st = 0; st < streams && ok; ++st) {
-            const int key0 = key_tile(it, st, j) * kPfN;
-            const int kvh = it.unit % p.kv_heads, bidx = it.unit / p.kv_heads;
-            for (int kv = 0; kv < 2; ++kv) {
-              const int s = u % C::kSlots;
-              if (u >= C::kSlots &&
-                  !(ok = mbar_wait(&kv_empty[s], ((u / C::kSlots) - 1) & 1,
-                                   kStatusTimeoutProducer)))
+        const int kvh = it.unit % p.kv_heads, bidx = it.unit / p.kv_heads;
+        if (!v_stream) {
+          // The Q buffer is free once every S of the previous busy item is done.
+          if (nq > 0 && !(ok = mbar_wait(q_empty, (nq - 1) & 1, kStatusTimeoutProducer))) break;
+          // Paired items share tile 0's Q.
+          const int qtiles = it.paired ? 1 : 2;
+          int ntiles = 0;
+          for (int t = 0; t < qtiles; ++t) ntiles += it.tile[t].nrows > 0 ? 1 : 0;
+          mbar_arrive_expect_tx(q_full, ntiles * C::kTileBytes);
+          for (int t = 0; t < qtiles; ++t)
+            if (it.tile[t].nrows > 0)
+              for (int c = 0; c < DCH; ++c)
+                tma_load_3d(sq + t * C::kTileBytes + c * C::kBoxBytes, &tm_q, q_full, c * 64,
+                            it.tile[t].row0, it.unit);
+          ++nq;
+        }
+        if (it.paired) {
+          // Stream order: (A, 0), (B, 0), (A, 1), ... (tile B may end first).
+          const int kv = v_stream ? 1 : 0;
+          const CUtensorMap* map = kv ? &tm_v : &tm_k;
+          for (int j = 0; j < it.j_count && ok; ++j)
+            for (int t = 0; t < 2; ++t) {
+              if (!tile_active(it, t, j)) continue;
+              const int s = kv * kHalf + u % kHalf;
+              if (u >= kHalf &&
+                  !(ok = mbar_wait(&kv_empty[s], ((u / kHalf) - 1) & 1, kStatusTimeoutProducer)))
                 break;
               uint8_t* dst = ring + s * C::kTileBytes;
               mbar_arrive_expect_tx(&kv_full[s], C::kTileBytes);
               for (int c = 0; c < DCH; ++c)
-                tma_load_4d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, &kv_full[s], c * 64,
-                            key0, kvh, bidx);
+                tma_load_4d(dst + c * C::kBoxBytes, map, &kv_full[s], c * 64,
+                            key_tile(it, t, j) * kPfN, kvh, bidx);
               ++u;
             }
+          continue;
+        }
+        for (int j = 0; j < it.j_count && ok; ++j) {
+          const int key0 = key_tile(it, 0, j) * kPfN;
+          for (int kv = 0; kv < 2; ++kv) {
+            const int s = u % C::kSlots;
+            if (u >= C::kSlots &&
+                !(ok = mbar_wait(&kv_empty[s], ((u / C::kSlots) - 1) & 1,
+                                 kStatusTimeoutProducer)))
+              break;
+            uint8_t* dst = ring + s * C::kTileBytes;
+            mbar_arrive_expect_tx(&kv_full[s], C::kTileBytes);
+            for (int c = 0; c < DCH; ++c)
+              tma_load_4d(dst + c * C::kBoxBytes, kv ? &tm_v : &tm_k, &kv_full[s], c * 64,
+                          key0, kvh, bidx);
+            ++u;
           }
         }
       }
       // Drain: never leave with copies in flight.
-      if (nq > 0) mbar_wait(q_full, (nq - 1) & 1, kStatusTimeoutProducer);
-      for (int v = max(0, u - C::kSlots); v < u; ++v)
-        mbar_wait(&kv_full[v % C::kSlots], (v / C::kSlots) & 1, kStatusTimeoutProducer);
+      if (!v_stream && nq > 0) mbar_wait(q_full, (nq - 1) & 1, kStatusTimeoutProducer);
+      if (kSplit && p.split_pairs) {
+        const int kv = v_stream ? 1 : 0;
+        for (int v = max(0, u - kHalf); v < u; ++v)
+          mbar_wait(&kv_full[kv * kHalf + v % kHalf], (v / kHalf) & 1, kStatusTimeoutProducer);
+      } else {
+        for (int v = max(0, u - C::kSlots); v < u; ++v)
+          mbar_wait(&kv_full[v % C::kSlots], (v / C::kSlots) & 1, kStatusTimeoutProducer);
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -366,7 +404,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       int n_act[2] = {0, 0};      // P tiles consumed per q tile (p_full phases)
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-        const PfItem it = prefill_item(p, ms, item);
+        const PfItem it = prefill_item<kSplit>(p, ms, item);
         if (!it.busy) continue;
         if (!(ok = mbar_wait(q_full, nq & 1, kStatusTimeoutMma))) break;
         ++nq;
@@ -404,36 +442,44 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         };
         bool first_pv[2] = {true, true};
         if (it.paired) {
-          // Each tile has its own K/V stream; every slot is released right
-          // after its only reader is issued.
-          auto pos = [&](int t, int j, int kv) { return paired_pos(it, t, j, kv); };
-          if (!(ok = wait_slot(pos(0, 0, 0)))) break;
-          issue_s_at(0, slot_addr(pos(0, 0, 0)));
-          release(pos(0, 0, 0));
+          // K and V sub-rings of kSlots / 2 slots, each filled in the order
+          // (A, 0), (B, 0), (A, 1), ...; every slot is released right after
+          // its only reader is issued.
+          constexpr int kHalf = C::kSlots / 2;
+          auto up = [&](int t, int j) { return ubase + j + min(j, it.kc[1]) + t; };
+          auto ps = [&](int kv, int pos) { return kv * kHalf + pos % kHalf; };
+          auto pwait = [&](int kv, int pos) {
+            return mbar_wait(&kv_full[ps(kv, pos)], (pos / kHalf) & 1, kStatusTimeoutMma);
+          };
+          auto paddr = [&](int kv, int pos) { return ring_addr + ps(kv, pos) * C::kTileBytes; };
+          auto prelease = [&](int kv, int pos) { mma_commit(&kv_empty[ps(kv, pos)]); };
+          if (!(ok = pwait(0, up(0, 0)))) break;
+          issue_s_at(0, paddr(0, up(0, 0)));
+          prelease(0, up(0, 0));
           if (tile_active(it, 1, 0)) {
-            if (!(ok = wait_slot(pos(1, 0, 0)))) break;
-            issue_s_at(1, slot_addr(pos(1, 0, 0)));
-            release(pos(1, 0, 0));
+            if (!(ok = pwait(0, up(1, 0)))) break;
+            issue_s_at(1, paddr(0, up(1, 0)));
+            prelease(0, up(1, 0));
           }
           for (int j = 0; j < it.j_count && ok; ++j) {
             for (int t = 0; t < 2 && ok; ++t) {
               if (!tile_active(it, t, j)) continue;
-              if (!(ok = wait_slot(pos(t, j, 1)))) break;  // V_t(j)
+              if (!(ok = pwait(1, up(t, j)))) break;  // V_t(j)
               if (!(ok = mbar_wait(&p_full[t], n_act[t] & 1, kStatusTimeoutMma))) break;
-              issue_pv_at(t, slot_addr(pos(t, j, 1)), first_pv[t]);
+              issue_pv_at(t, paddr(1, up(t, j)), first_pv[t]);
               first_pv[t] = false;
               ++n_act[t];
-              release(pos(t, j, 1));
+              prelease(1, up(t, j));
               if (tile_active(it, t, j + 1)) {
-                if (!(ok = wait_slot(pos(t, j + 1, 0)))) break;
-                issue_s_at(t, slot_addr(pos(t, j + 1, 0)));
-                release(pos(t, j + 1, 0));
+                if (!(ok = pwait(0, up(t, j + 1)))) break;
+                issue_s_at(t, paddr(0, up(t, j + 1)));
+                prelease(0, up(t, j + 1));
               }
             }
           }
           if (!ok) break;
           mma_commit(o_done);
-          ubase += paired_pos(it, 0, it.j_count, 0);
+          ubase += it.kc[0] + it.kc[1];
           continue;
         }
         auto issue_s = [&](int t, int j) { issue_s_at(t, slot_addr(2 * j)); };
@@ -515,9 +561,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     };
     int n_act0 = 0, n_act1 = 0;  // S tiles consumed per q tile (s_full phases)
     int n_done = 0;              // busy items finished (o_done phases)
+    int n_merge = 0;             // split tickets taken by this column half (part_done phases)
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-      const PfItem it = prefill_item(p, ms, item);
+      const PfItem it = prefill_item<kSplit>(p, ms, item);
       RowState st[2];
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
@@ -753,27 +800,26 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           bulk_commit();
         }
       };
-      for (int t = 0; t < 2; ++t) {
-        const TileInfo ti = t ? it.tile[1] : it.tile[0];
-        if (ti.nrows <= 0 || quarter * 32 >= ti.nrows || oc0 >= oc1) continue;
-        const RowState cs = t ? st[1] : st[0];
-        const float L = t ? lsum[1] : lsum[0];
-        const uint32_t o_tmem = tmem + lane_base + 256 + t * 128;
-        const bool have = cs.act > 0;
-        // O columns col .. col + 15 of this thread's row from TMEM (warp-collective).
-        auto load_o = [&](int col, float (&v)[16]) {
-          uint32_t ov[16];
-          tmem_ld16(o_tmem + col, ov);
-          tmem_ld_wait();
+      // O columns col .. col + 15 of this thread's row of tile t from TMEM
+      // (warp-collective).
+      auto load_o = [&](int t, int col, float (&v)[16]) {
+        uint32_t ov[16];
+        tmem_ld16(tmem + lane_base + 256 + t * 128 + col, ov);
+        tmem_ld_wait();
 #pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(ov[e]);
-        };
-        if (p.splits == 1) {
+        for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(ov[e]);
+      };
+      if constexpr (!kSplit) {
+        for (int t = 0; t < 2; ++t) {
+          const TileInfo ti = t ? it.tile[1] : it.tile[0];
+          if (ti.nrows <= 0 || quarter * 32 >= ti.nrows || oc0 >= oc1) continue;
+          const bool have = (t ? st[1].act : st[0].act) > 0;
+          const float L = t ? lsum[1] : lsum[0];
           const bool live = have && L > 0.f;
           const float inv = live ? 1.0f / L : 0.f;
           store_rows(ti, [&](int col, float (&v)[16]) {
             if (have) {
-              load_o(col, v);
+              load_o(t, col, v);
 #pragma unroll
               for (int e = 0; e < 16; ++e) v[e] = live ? v[e] * inv : 0.f;
             } else {
@@ -781,90 +827,168 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               for (int e = 0; e < 16; ++e) v[e] = 0.f;
             }
           });
-        } else {
-          // Split partial: O (unnormalised, this half's columns), m and l of
-          // this split; the warp that finishes a row group's last split
-          // merges all of them.  Paired items: both tiles are the same rows,
-          // splits it.split and it.split + 1.  m and l are kept per half, so
-          // each half's merge reads only what its own warps wrote.
+        }
+      } else {
+        // ---- key splits.  Each split leaves a partial per row: O
+        // (unnormalised, fp32), m and l, with m and l kept per column half so
+        // each half's merge reads only what its own warps wrote.  A paired
+        // item holds two splits of the same rows (tiles A and B), combined
+        // here first, so a row group has splits / 2 partials.  The four
+        // warps of a column half take one ticket per row group; in the CTA
+        // that brings the last partial they merge all of them, in partial
+        // order (deterministic), sharing the rows and columns between them.
+        const int np = it.paired ? p.splits / 2 : p.splits;
+        const int psplit = it.paired ? it.split / 2 : it.split;
+        for (int t = 0; t < (it.paired ? 1 : 2); ++t) {
+          const TileInfo ti = t ? it.tile[1] : it.tile[0];
+          if (ti.nrows <= 0) continue;  // the same for every warp
           const int ptile = it.paired ? it.pair_index : it.pair_index * 2 + t;
-          const int psplit = it.paired ? it.split + t : it.split;
-          const long long blk = (long long)ptile * p.splits;
-          float* po = p.ws_o + (blk + psplit) * (long long)p.d_pad * kPfM;
+          const long long blk = (long long)ptile * np;
+          auto po_of = [&](int sp) {
+            return reinterpret_cast<float4*>(p.ws_o + (blk + sp) * (long long)p.d_pad * kPfM);
+          };
           auto ml_of = [&](int sp) { return p.ws_ml + ((blk + sp) * 2 + h) * 2 * kPfM; };
-          // An empty split writes zeros, so the merge may read every partial.
-          for (int c0 = oc0; c0 < oc1; c0 += 16) {
-            float v[16];
-            if (have) {
-              load_o(c0, v);
-            } else {
+          if (quarter * 32 < ti.nrows && oc0 < oc1) {
+            // This row's tiles: t alone, or A and B rescaled to their common
+            // max.  A tile whose rows saw no key (act = 0, or m = -inf) adds
+            // nothing; an empty partial has m = -inf, l = 0 and O = 0.
+            const RowState& sa = t ? st[1] : st[0];
+            const bool use_b = it.paired;
+            const bool ha = sa.act > 0 && sa.m != -INFINITY;
+            const bool hb = use_b && st[1].act > 0 && st[1].m != -INFINITY;
+            float m = ha ? sa.m : -INFINITY;
+            if (hb) m = fmaxf(m, st[1].m);
+            const float wa = ha ? ex2(sa.m - m) : 0.f;
+            const float wb = hb ? ex2(st[1].m - m) : 0.f;
+            const float L = wa * (t ? lsum[1] : lsum[0]) + (use_b ? wb * lsum[1] : 0.f);
+            float4* po = po_of(psplit);
+            for (int c0 = oc0; c0 < oc1; c0 += 16) {
+              float v[16];
 #pragma unroll
               for (int e = 0; e < 16; ++e) v[e] = 0.f;
-            }
+              if (sa.act > 0) {  // warp-uniform
+                float a[16];
+                load_o(t, c0, a);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) po[(long long)(c0 + e) * kPfM + r] = v[e];
+                for (int e = 0; e < 16; ++e) v[e] = wa * a[e];
+              }
+              if (use_b && st[1].act > 0) {
+                float b[16];
+                load_o(1, c0, b);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] = fmaf(wb, b[e], v[e]);
+              }
+#pragma unroll
+              for (int g = 0; g < 4; ++g)
+                po[(c0 / 4 + g) * kPfM + r] =
+                    make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+            }
+            float* pml = ml_of(psplit);
+            pml[r] = ha || hb ? m : -INFINITY;
+            pml[kPfM + r] = L;
           }
-          float* pml = ml_of(psplit);
-          pml[r] = have ? cs.m : -INFINITY;
-          pml[kPfM + r] = have ? L : 0.f;
+          // The ticket: every thread's partial is visible device-wide before
+          // one thread of the half counts it (bounded waits: a warp that gave
+          // up elsewhere makes the others give up here, not hang).
           __threadfence();
-          __syncwarp();
-          unsigned int ticket = 0;
-          unsigned int* tk = p.tickets + (ptile * 4 + quarter) * 2 + h;
-          if (lane == 0) ticket = atomicAdd(tk, 1u);
-          ticket = __shfl_sync(0xffffffffu, ticket, 0);
-          if (ticket == (unsigned)p.splits - 1) {
-            __threadfence();
-            // Row max, then row sum, over the splits: eight splits' (m, l)
-            // loads in flight at a time (a split with m = -inf is empty).
-            float M = -INFINITY;
-            for (int sp0 = 0; sp0 < p.splits; sp0 += 8) {
-              float mv[8];
+          mbar_arrive(&part_done[h]);
+          const uint32_t mph = n_merge & 1;
+          ++n_merge;
+          unsigned int* tk = p.tickets + ptile * 2 + h;
+          if (quarter == 0 && lane == 0) {
+            int f = -1;
+            if (mbar_wait(&part_done[h], mph, kStatusTimeoutEpilogue))
+              f = atomicAdd(tk, 1u) == (unsigned)(np - 1) ? 1 : 0;
+            merge_flag[h] = f;
+            mbar_arrive(&flag_ready[h]);
+          }
+          const int flag = __all_sync(0xffffffffu, mbar_wait(&flag_ready[h], mph, kStatusTimeoutEpilogue))
+                               ? *(volatile int*)&merge_flag[h]
+                               : -1;
+          if (flag < 0) {
+            ok = false;
+            break;
+          }
+          const bool last = flag == 1;
+          if (!last) continue;
+          __threadfence();
+          if (quarter == 0 && lane == 0) atomicExch(tk, 0u);  // ready for the next call
+          // Work of this warp: row group rg (32 rows), column part `part`
+          // of this half (whole 16-column chunks).  Fewer than three row
+          // groups: the idle warps take column parts instead.
+          const int nq = (ti.nrows + 31) / 32;
+          const int parts = nq == 1 ? 4 : nq == 2 ? 2 : 1;
+          const int rg = parts == 1 ? quarter : quarter % nq;
+          const int part = parts == 1 ? 0 : quarter / nq;
+          const int nch = (oc1 - oc0) / 16;
+          const int cb = oc0 + 16 * (nch * part / parts);
+          const int ce = oc0 + 16 * (nch * (part + 1) / parts);
+          if (rg >= nq || cb >= ce) continue;
+          const int row = rg * 32 + lane;  // < 128: partial rows past nrows exist
+          // Row max and row sum over the partials in one pass, eight (m, l)
+          // loads in flight at a time; the sum is rescaled when a later batch
+          // raises the max.
+          float M = -INFINITY, Ls = 0.f;
+          for (int sp0 = 0; sp0 < np; sp0 += 8) {
+            float mv[8], lv[8];
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                mv[i] = sp0 + i < p.splits ? __ldcg(ml_of(sp0 + i) + r) : -INFINITY;
-#pragma unroll
-              for (int i = 0; i < 8; ++i) M = fmaxf(M, mv[i]);
+            for (int i = 0; i < 8; ++i) {
+              const bool in = sp0 + i < np;
+              mv[i] = in ? __ldcg(ml_of(sp0 + i) + row) : -INFINITY;
+              lv[i] = in ? __ldcg(ml_of(sp0 + i) + kPfM + row) : 0.f;
             }
-            float Ls = 0.f;
-            for (int sp0 = 0; sp0 < p.splits; sp0 += 8) {
-              float mv[8], lv[8];
+            float mb = M;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mb = fmaxf(mb, mv[i]);
+            if (mb != -INFINITY) {
+              if (M != -INFINITY) Ls *= ex2(M - mb);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) Ls += mv[i] == -INFINITY ? 0.f : ex2(mv[i] - mb) * lv[i];
+              M = mb;
+            }
+          }
+          const float inv = Ls > 0.f ? 1.0f / Ls : 0.f;
+          __nv_bfloat16* orow = p.o + ((long long)it.unit * p.rows + ti.row0 + row) * p.head_dim;
+          for (int col = cb; col < ce; col += 16) {
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = 0.f;
+            // Eight partials per batch: their m and O loads all in flight
+            // together (past the last partial the loads read partial 0 with
+            // weight 0).
+            for (int sp0 = 0; sp0 < np; sp0 += 8) {
+              float mv[8];
+              float x8[8][16];
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const bool in = sp0 + i < p.splits;
-                mv[i] = in ? __ldcg(ml_of(sp0 + i) + r) : -INFINITY;
-                lv[i] = in ? __ldcg(ml_of(sp0 + i) + kPfM + r) : 0.f;
+                const int sp = sp0 + i < np ? sp0 + i : 0;
+                mv[i] = sp0 + i < np ? __ldcg(ml_of(sp) + row) : -INFINITY;
+                const float4* src = po_of(sp) + row;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                  const float4 f = __ldcg(src + (col / 4 + g) * kPfM);
+                  x8[i][4 * g] = f.x;
+                  x8[i][4 * g + 1] = f.y;
+                  x8[i][4 * g + 2] = f.z;
+                  x8[i][4 * g + 3] = f.w;
+                }
               }
 #pragma unroll
-              for (int i = 0; i < 8; ++i) Ls += mv[i] == -INFINITY ? 0.f : ex2(mv[i] - M) * lv[i];
+              for (int i = 0; i < 8; ++i) {
+                const float w = mv[i] == -INFINITY ? 0.f : ex2(mv[i] - M) * inv;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] = fmaf(w, x8[i][e], v[e]);
+              }
             }
-            const float inv = Ls > 0.f ? 1.0f / Ls : 0.f;
-            store_rows(ti, [&](int col, float (&v)[16]) {
+            if (row < ti.nrows) {
+              // 8 columns (16 bytes) at a time; head_dim is a multiple of 8.
 #pragma unroll
-              for (int e = 0; e < 16; ++e) v[e] = 0.f;
-              // Four splits per batch: their m and O loads all in flight
-              // together (every partial was written; past the last split the
-              // loads read split 0 with weight 0).
-              for (int sp0 = 0; sp0 < p.splits; sp0 += 4) {
-                float mv[4];
-                float x4[4][16];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const int sp = sp0 + i < p.splits ? sp0 + i : 0;
-                  mv[i] = sp0 + i < p.splits ? __ldcg(ml_of(sp) + r) : -INFINITY;
-                  const float* src = p.ws_o + (blk + sp) * (long long)p.d_pad * kPfM + r;
-#pragma unroll
-                  for (int e = 0; e < 16; ++e) x4[i][e] = __ldcg(src + (long long)(col + e) * kPfM);
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const float w = mv[i] == -INFINITY ? 0.f : ex2(mv[i] - M) * inv;
-#pragma unroll
-                  for (int e = 0; e < 16; ++e) v[e] = fmaf(w, x4[i][e], v[e]);
-                }
-              }
-            });
-            if (lane == 0) atomicExch(tk, 0u);  // ready for the next call
+              for (int g = 0; g < 2; ++g)
+                if (col + 8 * g < p.head_dim)
+                  *reinterpret_cast<uint4*>(orow + col + 8 * g) =
+                      make_uint4(pack_bf16(v[8 * g], v[8 * g + 1]), pack_bf16(v[8 * g + 2], v[8 * g + 3]),
+                                 pack_bf16(v[8 * g + 4], v[8 * g + 5]), pack_bf16(v[8 * g + 6], v[8 * g + 7]));
+            }
           }
         }
       }
