@@ -131,7 +131,10 @@ int gqa_attn_describe(int batch, int q_len, int kv_len, int num_q_heads, int num
  * key 1: force the path (value 0 = automatic, 1 = decode, 2 = prefill);
  * key 2: force the number of key tiles per decode split (0 = automatic);
  * key 3: force the number of key splits of the tcgen05 kernel for units with
- *        one row tile (rounded up to even; 0 = automatic).
+ *        one row tile (rounded up to even; 0 = automatic);
+ * key 4: how those splits merge (0 = automatic: through distributed shared
+ *        memory in one thread-block cluster per unit when the whole grid fits
+ *        on the device at once; -1 = always through the workspace).
  * A forced path that cannot run these sizes falls back to automatic.
  * Returns GQA_ATTN_OK or GQA_ATTN_ERR_ARG for an unknown key.
  */

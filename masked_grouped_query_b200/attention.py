@@ -134,9 +134,11 @@ def describe(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, causal=F
 
 def set_override(key: str, value: int) -> None:
     """Test/tuning knob: ``force_path`` (0 auto, 1 decode, 2 prefill),
-    ``tiles_per_split`` (decode, 0 = automatic) or ``prefill_splits``
-    (tcgen05 kernel, units with one row tile; 0 = automatic)."""
-    k = {"force_path": 1, "tiles_per_split": 2, "prefill_splits": 3}[key]
+    ``tiles_per_split`` (decode, 0 = automatic), ``prefill_splits``
+    (tcgen05 kernel, units with one row tile; 0 = automatic) or
+    ``prefill_cluster`` (how those splits merge: 0 automatic, -1 always
+    through the workspace instead of a thread-block cluster)."""
+    k = {"force_path": 1, "tiles_per_split": 2, "prefill_splits": 3, "prefill_cluster": 4}[key]
     _lib.check(_lib.load().gqa_attn_set_override(k, int(value)), "gqa_attn_set_override")
 
 

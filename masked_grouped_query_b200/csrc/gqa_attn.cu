@@ -37,12 +37,20 @@ struct DeviceInfo {
   int smem_optin = 0;
   bool decode_attr[8] = {false, false, false, false, false, false, false, false};
   bool prefill_attr[12] = {};  // per (DCH, softcap degree, split) instantiation
+  // Clusters of n CTAs of a split instantiation that can be resident at once
+  // (cudaOccupancyMaxActiveClusters); -1 = not asked yet.
+  int cluster_max[12][9];
+  DeviceInfo() {
+    for (auto& a : cluster_max)
+      for (int& n : a) n = -1;
+  }
 };
 
 std::mutex g_mu;
 DeviceInfo g_dev[64];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::atomic<int> g_force_path{0};
+std::atomic<int> g_no_cluster{0};
 std::atomic<int> g_force_tps{0};
 std::atomic<int> g_force_pf_splits{0};
 
@@ -520,12 +528,62 @@ int launch_prefill_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.tickets = (unsigned int*)tickets;
   p.pair_heads = pl.pair_heads;
   p.heavy_first = (pr.causal || pr.window > 0) && !pl.split_pairs ? 1 : 0;
+  // Paired key splits, one item per CTA: a cluster per unit merges its
+  // partials through distributed shared memory, when every cluster of the
+  // grid can be resident at once (one wave); otherwise the workspace merge.
+  int csize = 0;
+  if (kSplit && pl.split_pairs && !g_no_cluster.load()) {
+    const int half = pl.splits / 2;
+    if (half >= 2 && half <= 8 && pl.ctas == pr.units * half) {
+      int& fit = dev.cluster_max[attr][half];
+      if (fit < 0) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute at[1];
+        at[0].id = cudaLaunchAttributeClusterDimension;
+        at[0].val.clusterDim.x = (unsigned)half;
+        at[0].val.clusterDim.y = 1;
+        at[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3((unsigned)pl.ctas);
+        cfg.blockDim = dim3(kPfThreads);
+        cfg.dynamicSmemBytes = C::kSmemBytes;
+        cfg.attrs = at;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, prefill_sm100_kernel<DCH, kCapDeg, kSplit>, &cfg) !=
+            cudaSuccess) {
+          (void)cudaGetLastError();
+          n = 0;
+        }
+        fit = n;
+      }
+      if (fit >= pr.units) csize = half;
+    }
+  }
+  p.cluster_merge = csize;
   p.causal = pr.causal;
   p.window = pr.window;
   const float rs = 1.0f / std::sqrt((float)pr.d);
   p.logit_scale = kLog2e * rs;
   p.cap_in = kCap ? rs / pr.softcap : 0.f;
   p.cap_out = kCap ? pr.softcap * kLog2e : 0.f;
+  if (csize > 0) {
+    // One item per CTA, clusters of csize consecutive CTAs (one unit each).
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)csize;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)pl.ctas);
+    cfg.blockDim = dim3(kPfThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    const cudaError_t e =
+        cudaLaunchKernelEx(&cfg, prefill_sm100_kernel<DCH, kCapDeg, kSplit>, tq, tk, tv, to, p);
+    return e == cudaSuccess ? GQA_ATTN_OK : cuda_fail("launch(prefill, clusters)", e, GQA_ATTN_ERR_LAUNCH);
+  }
   // Persistent: at most one CTA per SM, each walking items with stride grid.
   const int grid = (int)(pl.ctas < dev.sms ? pl.ctas : dev.sms);
   prefill_sm100_kernel<DCH, kCapDeg, kSplit><<<dim3((unsigned)grid), kPfThreads, C::kSmemBytes, stream>>>(
@@ -733,6 +791,10 @@ int gqa_attn_set_override(int key, int value) {
   }
   if (key == 3) {
     g_force_pf_splits.store(value > 0 ? value : 0);
+    return GQA_ATTN_OK;
+  }
+  if (key == 4) {
+    g_no_cluster.store(value < 0 ? 1 : 0);
     return GQA_ATTN_OK;
   }
   return GQA_ATTN_ERR_ARG;

@@ -75,6 +75,9 @@ struct PrefillParams {
   int n_items;           // units * pairs_per_unit * splits (/ 2 when split_pairs)
   int pair_heads;        // 1: tiles (2p, 2p+1) are two heads at one position
   int heavy_first;       // 1: items run in order of decreasing key-tile count (causal / window)
+  int cluster_merge;     // paired items, one per CTA, launched as clusters of this many CTAs
+                         // (one cluster per unit): partials merge through distributed
+                         // shared memory instead of the workspace; 0 = workspace merge
   int causal, window;
   float logit_scale, cap_in, cap_out;
   // Split partials (splits > 1): per (pair, tile, split) O as fp32
@@ -346,6 +349,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (it.paired) {
           // Stream order: (A, 0), (B, 0), (A, 1), ... (tile B may end first).
           const int kv = v_stream ? 1 : 0;
+          // At the start every CTA asks for its first tiles at once; V is
+          // needed one softmax later than Q and K, so it queues behind them.
+          if (v_stream && u == 0 &&
+              !(ok = mbar_wait(&kv_full[0], 0, kStatusTimeoutProducer)))
+            break;
           const CUtensorMap* map = kv ? &tm_v : &tm_k;
           for (int j = 0; j < it.j_count && ok; ++j)
             for (int t = 0; t < 2; ++t) {
@@ -848,6 +856,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             return reinterpret_cast<float4*>(p.ws_o + (blk + sp) * (long long)p.d_pad * kPfM);
           };
           auto ml_of = [&](int sp) { return p.ws_ml + ((blk + sp) * 2 + h) * 2 * kPfM; };
+          // Cluster merge: the combined partial stays in this CTA's shared
+          // memory (the K/V ring and staging area are idle after the CTA's
+          // only item): O as fp32 rows of d_pad + 4 floats, m and l per row.
+          const bool to_smem = it.paired && p.cluster_merge > 0;
           if (quarter * 32 < ti.nrows && oc0 < oc1) {
             // This row's tiles: t alone, or A and B rescaled to their common
             // max.  A tile whose rows saw no key (act = 0, or m = -inf) adds
@@ -862,6 +874,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const float wb = hb ? ex2(st[1].m - m) : 0.f;
             const float L = wa * (t ? lsum[1] : lsum[0]) + (use_b ? wb * lsum[1] : 0.f);
             float4* po = po_of(psplit);
+            float* crow = reinterpret_cast<float*>(ring) + r * (p.d_pad + 4);
             for (int c0 = oc0; c0 < oc1; c0 += 16) {
               float v[16];
 #pragma unroll
@@ -879,14 +892,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 for (int e = 0; e < 16; ++e) v[e] = fmaf(wb, b[e], v[e]);
               }
 #pragma unroll
-              for (int g = 0; g < 4; ++g)
-                po[(c0 / 4 + g) * kPfM + r] =
-                    make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+              for (int g = 0; g < 4; ++g) {
+                const float4 f = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
+                if (to_smem)
+                  *reinterpret_cast<float4*>(crow + c0 + 4 * g) = f;
+                else
+                  po[(c0 / 4 + g) * kPfM + r] = f;
+              }
             }
-            float* pml = ml_of(psplit);
-            pml[r] = ha || hb ? m : -INFINITY;
-            pml[kPfM + r] = L;
+            float* pml = to_smem ? reinterpret_cast<float*>(stage_all) : ml_of(psplit);
+            if (!to_smem || h == 0) {
+              pml[r] = ha || hb ? m : -INFINITY;
+              pml[kPfM + r] = L;
+            }
           }
+          if (to_smem) continue;  // merged after the cluster barrier
           // The ticket: every thread's partial is visible device-wide before
           // one thread of the half counts it (bounded waits: a warp that gave
           // up elsewhere makes the others give up here, not hang).
@@ -994,6 +1014,69 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       }
     }
     if (lane == 0) bulk_wait_all();  // stores done before the CTA exits
+  }
+
+  // ---------------------------------------------------------------- cluster merge
+  // Every thread of every CTA reaches both cluster barriers (no role leaves
+  // the kernel early; all waits above are bounded).  Between them the
+  // softmax warps of CTA `rank` merge column groups [g0, g1) of every row
+  // from the partials of all CTAs of the cluster, in rank order.
+  if constexpr (kSplit) {
+    if (p.cluster_merge > 0) {
+      __syncwarp();
+      cluster_sync();
+      if (warp >= 4) {
+        const int csize = p.cluster_merge;
+        const uint32_t rank = cluster_ctarank();
+        const int G = p.d_pad / 4;
+        const int g0 = (int)rank * G / csize, g1 = ((int)rank + 1) * G / csize, ng = g1 - g0;
+        const int nrows = min(kPfM, p.rows);
+        const int unit = (int)blockIdx.x / csize;
+        const int stride = p.d_pad + 4;
+        const float* cpart = reinterpret_cast<const float*>(ring);
+        const float* cml = reinterpret_cast<const float*>(stage_all);
+        for (int i = threadIdx.x - 128; i < nrows * ng; i += 256) {
+          const int row = i / ng, g = g0 + i % ng;
+          // Every peer's m, l and O values of this row and column group,
+          // all loads in flight together; then the weighted sum in rank order.
+          float mv[8], lv[8];
+          float4 f[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            mv[c] = -INFINITY;
+            lv[c] = 0.f;
+            f[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c < csize) {
+              mv[c] = ld_dsmem(dsmem_addr(cml + row, c));
+              lv[c] = ld_dsmem(dsmem_addr(cml + kPfM + row, c));
+              f[c] = ld_dsmem_v4(dsmem_addr(cpart + row * stride + 4 * g, c));
+            }
+          }
+          float M = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) M = fmaxf(M, mv[c]);
+          float Ls = 0.f;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float w = mv[c] == -INFINITY ? 0.f : ex2(mv[c] - M);
+            Ls = fmaf(w, lv[c], Ls);
+            acc.x = fmaf(w, f[c].x, acc.x);
+            acc.y = fmaf(w, f[c].y, acc.y);
+            acc.z = fmaf(w, f[c].z, acc.z);
+            acc.w = fmaf(w, f[c].w, acc.w);
+          }
+          const float inv = Ls > 0.f ? 1.0f / Ls : 0.f;
+          if (4 * g < p.head_dim) {  // head_dim is a multiple of 8
+            __nv_bfloat16* dst = p.o + ((long long)unit * p.rows + row) * p.head_dim + 4 * g;
+            *reinterpret_cast<uint2*>(dst) =
+                make_uint2(pack_bf16(acc.x * inv, acc.y * inv), pack_bf16(acc.z * inv, acc.w * inv));
+          }
+        }
+      }
+      __syncwarp();
+      cluster_sync();  // the peers have read this CTA's partial
+    }
   }
 
   // ---------------------------------------------------------------- teardown

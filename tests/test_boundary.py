@@ -128,6 +128,18 @@ def test_ring_rejects_bad_arguments_without_a_device(lib):
     assert _ring(lib, flags=0x1) == -7
 
 
+def test_override_keys(lib):
+    # Keys 1-4 are knobs (host state only, no device needed); others are rejected.
+    for key in (1, 2, 3, 4):
+        assert lib.gqa_attn_set_override(key, 0) == 0
+    assert lib.gqa_attn_set_override(4, -1) == 0
+    assert lib.gqa_attn_set_override(4, 0) == 0
+    assert lib.gqa_attn_set_override(5, 0) == -12  # GQA_ATTN_ERR_ARG
+    assert lib.gqa_attn_set_override(0, 0) == -12
+    with pytest.raises(KeyError):
+        mgq.set_override("no_such_knob", 1)
+
+
 def test_no_device_means_device_error(lib):
     if torch.cuda.is_available():
         pytest.skip("a CUDA device is present")

@@ -219,6 +219,36 @@ def test_tcgen05_key_splits(cfg):
     assert torch.equal(a, b2)  # deterministic merge order
 
 
+@pytest.mark.parametrize("cfg", [
+    (8, 4, 32768, 64, 4, 128, True, 4096, 30.0),   # 4 CTAs per unit
+    (1, 3, 1000, 16, 1, 72, False, 300, None),     # 2 CTAs per unit, D = 72
+    (3, 2, 777, 32, 2, 64, True, None, 20.0),      # 4 CTAs per unit, D = 64
+])
+def test_paired_split_merges(cfg):
+    # Units with one row tile take two key splits per CTA; the partials
+    # merge through a cluster's distributed shared memory (automatic) or
+    # through the workspace (forced).  Both against the oracle, each
+    # deterministic, and the two within rounding of each other.
+    b, lq, lk, hq, hkv, d, causal, window, cap = cfg
+    w = Workload("pm", b, lq, lk, hq, hkv, d, causal, window, cap, seed=lk + 3 * d)
+    q, k, v = make_inputs(w)
+    want = oracle.attention(q, k, v, causal=causal, window=window, softcap=cap)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    outs = []
+    try:
+        for mode in (0, -1):
+            mgq.set_override("prefill_cluster", mode)
+            a = mgq.attention(q, k, v, causal=causal, window=window, softcap=cap)
+            a2 = mgq.attention(q, k, v, causal=causal, window=window, softcap=cap)
+            torch.cuda.synchronize()
+            assert torch.equal(a, a2)
+            assert_close(a, want, f"merge mode {mode}")
+            outs.append(a.float())
+    finally:
+        mgq.set_override("prefill_cluster", 0)
+    assert (outs[0] - outs[1]).abs().max().item() <= 2.0 ** -6
+
+
 def test_host_buffer_entry_point_matches_device_entry_point():
     w = Workload("h", 2, 3, 333, 8, 2, 128, True, 100, 30.0, 21)
     q, k, v = make_inputs(w)
