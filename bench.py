@@ -28,6 +28,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import subprocess
 import sys
 import time
@@ -102,13 +103,28 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+_CODE_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|//[^\n]*|/\*.*?\*/|\s+', re.S)
+
+
+def _strip_comments(text: str) -> str:
+    """C/CUDA source with comments removed and whitespace runs collapsed
+    (string literals kept), so edits to comments alone keep the hash."""
+    def sub(m):
+        t = m.group(0)
+        return t if t.startswith('"') else " "
+    return _CODE_TOKENS.sub(sub, text).strip()
+
+
 def kernel_source_hash() -> str:
+    """Hash of the kernel sources' code (not their comments): the ncu figures
+    in profiles/traffic.json are reported only while it matches."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "masked_grouped_query_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                code = _strip_comments(f.read())
+            h.update(name.encode() + b"\0" + code.encode())
     return h.hexdigest()[:16]
 
 

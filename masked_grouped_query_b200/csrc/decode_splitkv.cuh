@@ -3,12 +3,13 @@
 //
 // Work unit: one kv head of one batch element (b, kvh) and a block of up to
 // 64 "rows" -- the q rows of every q head of that GQA group, packed so each
-// K/V tile feeds all of them ("north star" (3); the grouped-query decode step
+// K/V tile feeds all of them (the decode shapes with GQA ratios 1:1 to 16:1
 // of "TPU v6e Masked GQA Kernel Optimization", "What You Have").  The key
 // range of a row block is cut into `splits` chunks; one CTA per chunk.
 //
 // Per CTA: one loader warp streams 64-key K and V tiles with TMA
-// (cp.async.bulk.tensor, 128-byte swizzle) into a 4-stage mbarrier ring;
+// (cp.async.bulk.tensor, 128-byte swizzle) into a ring of 3 stages (2 for
+// head_dim above 128) guarded by mbarriers;
 // four compute warps run S = Q K^T and O += P V on the tensor cores with
 // mma.sync m16n8k16 (bf16 in, fp32 accumulate) and an online fp32 softmax
 // with the softcap and mask fused in.  Chunks end with a log-sum-exp partial

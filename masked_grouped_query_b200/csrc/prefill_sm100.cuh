@@ -6,8 +6,9 @@
 // cut into 128-row tiles.  A work item is a pair of tiles whose key ranges
 // coincide or overlap (two heads of the group at the same positions when
 // q_len is a multiple of 128, else two consecutive tiles), so every K/V tile
-// loaded for the item feeds both ("north star" (2): the q heads of a GQA
-// group are packed so each K/V tile is read once).
+// loaded for the item feeds both: the q heads of a GQA group share one kv
+// head ("TPU v6e Masked GQA Kernel Optimization", "What You Have": GQA
+// ratios 1:1 to 16:1), so its K/V tiles are read once for all of them.
 //
 // Persistent: one CTA per SM walks the items blockIdx.x, blockIdx.x +
 // gridDim.x, ...; TMEM, barriers and the K/V ring live across items, and the
