@@ -103,7 +103,7 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-_CODE_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|//[^\n]*|/\*.*?\*/|\s+', re.S)
+_CODE_TOKENS = re.compile(r'"(?:\\.|[^"\\\n])*"|(?:\s|//[^\n]*|/\*.*?\*/)+', re.S)
 
 
 def _strip_comments(text: str) -> str:
@@ -115,11 +115,11 @@ def _strip_comments(text: str) -> str:
     return _CODE_TOKENS.sub(sub, text).strip()
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(csrc: str | None = None) -> str:
     """Hash of the kernel sources' code (not their comments): the ncu figures
     in profiles/traffic.json are reported only while it matches."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "masked_grouped_query_b200", "csrc")
+    csrc = csrc or os.path.join(ROOT, "masked_grouped_query_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh")):
             with open(os.path.join(csrc, name), encoding="utf-8") as f:
