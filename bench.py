@@ -548,13 +548,13 @@ def main():
             extra[st.name] = {"metric": "decode step on a KV cache (append + attend) GB/s",
                               "value": a, "unit": "GB/s", "ms": r["ms_mean"],
                               "frac_of_peak": a / pk["hbm_gbs"], "launches_per_step": 1}
-        for name, rs in RING_STEPS.items():
+        for ring_name, rs in RING_STEPS.items():
             r = time_ring(rs, max(20, args.steps // 4), args.warmup, device)
             a = r["bytes"] / 1e9 / (r["ms_mean"] * 1e-3)
-            extra[name] = {"metric": "masked-GQA attn fwd KV-read GB/s (decode, ring window)",
-                           "value": a, "unit": "GB/s", "ms": r["ms_mean"],
-                           "frac_of_peak": a / pk["hbm_gbs"],
-                           "shape": {k: v for k, v in rs.items() if k != "seed"}}
+            extra[ring_name] = {"metric": "masked-GQA attn fwd KV-read GB/s (decode, ring window)",
+                                "value": a, "unit": "GB/s", "ms": r["ms_mean"],
+                                "frac_of_peak": a / pk["hbm_gbs"],
+                                "shape": {k: v for k, v in rs.items() if k != "seed"}}
         r = time_kv_append(2, 4096, 4, 128, 4096, max(20, args.steps // 4), args.warmup, device)
         a = r["bytes"] / 1e9 / (r["ms_mean"] * 1e-3)
         extra["kv_append_prompt_block"] = {
