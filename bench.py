@@ -385,6 +385,18 @@ def time_e2e(w: Workload, steps: int, warmup: int, device):
 
 
 # ------------------------------------------------------------ oracle arm
+def cpu_model() -> str:
+    """The host CPU's model name (Linux /proc/cpuinfo), or "" when unknown."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return ""
+
+
 def cpu_sample(w: Workload, budget_s: float = 12.0):
     """Time the oracle on whole kv-head groups of the workload; returns
     (metric value, sample description, threads, seconds)."""
@@ -507,7 +519,7 @@ def main():
                 "dtype": "f64", "data": "synthetic",
                 "config": {"workload": w.name, **{k: v for k, v in w.cfg().items() if k not in ("name",)}},
                 "cpu_baseline": {"value": value, "unit": unit, "cores": threads,
-                                 "kind": "oracle", "sample": desc},
+                                 "kind": "oracle", "sample": desc, "cpu": cpu_model()},
                 "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
@@ -595,7 +607,7 @@ def main():
         if ctx.world == 1 and not args.no_cpu:
             val, desc, threads, _ = cpu_sample(w)
             line["cpu_baseline"] = {"value": val, "unit": unit, "cores": threads,
-                                    "kind": "oracle", "sample": desc}
+                                    "kind": "oracle", "sample": desc, "cpu": cpu_model()}
         if extra:
             line["other_workloads"] = extra
         print(json.dumps(line))
