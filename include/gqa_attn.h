@@ -86,10 +86,15 @@ extern "C" {
  *
  * The call validates, plans and enqueues 1 kernel (a memset when kv_len == 0,
  * nothing when o is empty) on `stream` and returns without synchronising.
- * Split-KV decode partials live in a library-owned workspace per (device,
- * stream), allocated with cudaMalloc on first need and grown on demand (so
- * the first call of a new size synchronises the device); calls on one
- * stream are ordered, calls on different streams do not share workspace.
+ * Key-split partials live in a library-owned workspace per (device, stream),
+ * allocated with cudaMalloc on first need and grown on demand (so the first
+ * call of a new size synchronises the device); calls on one stream are
+ * ordered, calls on different streams do not share workspace.  Partials of
+ * the split-KV decode kernel and of the tcgen05 kernel's key splits use it;
+ * when every (batch, kv head) has one 128-row tile and its CTAs fit on the
+ * device at once, the tcgen05 kernel is launched as one thread-block cluster
+ * per (batch, kv head) and merges its partials in distributed shared memory
+ * instead.
  *
  * Returns GQA_ATTN_OK or a negative GQA_ATTN_ERR_* code.  Errors raised while
  * the kernel runs surface at the next synchronisation (CUDA convention) and,
@@ -118,8 +123,9 @@ int gqa_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host
  * the current device, without launching anything.  Any output pointer may
  * be NULL.  *path: 0 = nothing to do, 1 = split-KV decode kernel, 2 = tcgen05
  * prefill kernel, 3 = zero fill (kv_len == 0).  *splits: key chunks per row
- * block (decode) or 1.  *ctas: CTAs of the launch.  *tiles: key tiles of the
- * widest row block.  Returns GQA_ATTN_OK or the error gqa_attn_fwd would
+ * block (decode) or key-range splits per row tile (tcgen05 kernel; 1 = none).
+ * *ctas: work items of the launch (CTAs, or items of the persistent grid).
+ * *tiles: key tiles of the widest row block.  Returns GQA_ATTN_OK or the error gqa_attn_fwd would
  * return for these sizes.
  */
 int gqa_attn_describe(int batch, int q_len, int kv_len, int num_q_heads, int num_kv_heads,
