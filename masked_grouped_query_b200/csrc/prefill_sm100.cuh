@@ -26,24 +26,25 @@
 //               N = head_dim rounded up to 16);
 //   warps 2-3   idle but for warp 2's V stream of paired items (they
 //               complete warpgroup 0 for the register split);
-//   warps 4-11  softmax + epilogue: warps 4-7 take key columns [0, 64) of
-//               each S tile, warps 8-11 columns [64, 128).  A thread owns
-//               half of one row: it reads that half from TMEM, applies
-//               scale, softcap and mask, and swaps its partial row max with
-//               the partner thread (same TMEM lane, other half) through
-//               shared memory under a named barrier; both then keep the same
-//               running max (online softmax, rescaling their halves of O in
-//               TMEM only when the max grows by more than 2^8), write P as
-//               bf16 back over S in TMEM and keep half-row sums, added up at
-//               the end of the item, when each half normalises and stores
-//               its half of the O row.
-// The eight softmax warps take tile A, then tile B, at every key step: while
-// they work on one tile the tensor core runs the other tile's P.V and next
-// S, and two warps per SM sub-partition share each softmax.
+//   warps 4-7   softmax + epilogue of q tile A, warps 8-11 of q tile B: a
+//               thread owns one row of its tile.  It reads the row's 128
+//               scores of an S tile from TMEM, applies scale, softcap and
+//               mask, keeps the running max and sum in fp32 (online softmax,
+//               rescaling its O row in TMEM only when the max grows by more
+//               than 2^8), writes P as bf16 back over S in TMEM, and at the
+//               end of the item normalises its O row and stores it.
+// The two softmax warpgroups work on their own tiles at the same time, out
+// of phase: while one computes its softmax the tensor core runs the other
+// tile's P.V and next S, and the two warps each SM sub-partition holds (one
+// per tile) hide each other's waits.  Of every 32 scores of a row, a fixed
+// share takes 2^x from a polynomial on the FMA pipe instead of the MUFU
+// unit, so the two pipes share the exponentials.
 //
 // Fully masked key tiles are never loaded; tiles wholly inside every row's
 // visible range skip the per-element mask.  All waits are bounded.
 #pragma once
+
+#include <type_traits>
 
 #include "mask.cuh"
 #include "ptx.cuh"
@@ -58,10 +59,13 @@ constexpr int kPfThreads = 32 * kPfWarps;
 // the two softmax warpgroups rise to kRegsHigh.  The host checks before every
 // launch that 4*32*kRegsLow + 8*32*kRegsHigh fits in the registers the block
 // is launched with, so the increase can always be granted.
-constexpr int kRegsLow = 96;
-constexpr int kRegsHigh = 200;
+constexpr int kRegsLow = 88;
+constexpr int kRegsHigh = 208;
 constexpr int kRegSplitTotal = 4 * 32 * kRegsLow + 8 * 32 * kRegsHigh;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+// Of every 16 score pairs (32 keys) of a row, pairs [kEmuFrom, 16) take 2^x
+// from exp2_poly_x2 (FMA pipe) on tiles without a mask, the rest from MUFU.
+constexpr int kEmuFrom = 12;
 
 struct PrefillParams {
   __nv_bfloat16* o;
@@ -99,12 +103,14 @@ struct PrefillCfg {
   static constexpr int kRingBytes = kSlots * kTileBytes;
   // Output staging: one 32-row x 64-column bf16 box (4 KB) per softmax warp.
   static constexpr int kStageBytes = 8 * 4096;
-  // Row values swapped between the two column halves: [half][row] fp32.
-  static constexpr int kXchgBytes = 2 * 128 * 4;
-  static constexpr int kBarOffset = kQBytes + kRingBytes + kStageBytes + kXchgBytes;
-  // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done, drain,
-  // part_done[2], flag_ready[2]
-  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 1 + 1 + 2 + 2;
+  // (m, l) of a row swapped between the two softmax warpgroups (paired key
+  // splits, which write no output through the staging boxes):
+  // [warpgroup][row] float2 at this offset in the staging area.
+  static constexpr int kXchgOffset = 16384;
+  static constexpr int kBarOffset = kQBytes + kRingBytes + kStageBytes;
+  // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2],
+  // drain, part_done[2], flag_ready[2]
+  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 1 + 2 + 2;
   static constexpr int kSmemBytes = 1024 + kBarOffset + kNumBars * 8 + 16;
 };
 
@@ -260,7 +266,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint8_t* sq = smem;                   // Q tiles A, B
   uint8_t* ring = smem + C::kQBytes;    // K/V slots
   uint8_t* stage_all = ring + C::kRingBytes;  // output staging, 4 KB per softmax warp
-  float* xchg = (float*)(stage_all + C::kStageBytes);
+  float2* xchg = (float2*)(stage_all + C::kXchgOffset);
   uint64_t* bars = (uint64_t*)(smem + C::kBarOffset);
   uint64_t* q_full = bars;
   uint64_t* q_empty = bars + 1;
@@ -268,10 +274,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   uint64_t* kv_empty = kv_full + C::kSlots;
   uint64_t* s_full = kv_empty + C::kSlots;
   uint64_t* p_full = s_full + 2;
-  uint64_t* o_done = p_full + 2;  // every MMA of an item has finished
-  uint64_t* drain = o_done + 1;
-  // Key splits: the four warps of a column half have written their partials
-  // (part_done[h]), and the ticket's answer is in merge_flag[h] (flag_ready[h]).
+  uint64_t* o_done = p_full + 2;  // [t]: every MMA of q tile t in the item has finished
+  uint64_t* drain = o_done + 2;
+  // Key splits: the four warps of softmax warpgroup t have written their
+  // partials (part_done[t]), and the ticket's answer is in merge_flag[t]
+  // (flag_ready[t]).
   uint64_t* part_done = drain + 1;
   uint64_t* flag_ready = part_done + 2;
   uint32_t* tmem_slot = (uint32_t*)(flag_ready + 2);
@@ -289,9 +296,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 256);
+      mbar_init(&p_full[t], 4);  // one arrival per warp of the tile's warpgroup
+      mbar_init(&o_done[t], 1);
     }
-    mbar_init(o_done, 1);
     mbar_init(drain, 1);
     for (int t = 0; t < 2; ++t) {
       mbar_init(&part_done[t], 128);
@@ -308,7 +315,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   // TMEM columns: S_A [0,128), S_B [128,256), O_A [256,384), O_B [384,512).
-  // P_t (bf16 pairs) overwrites the first 64 columns of S_t.
+  // P_t (bf16 pairs) overwrites the first 64 columns of S_t.  Named barriers
+  // 1 + q (64 threads): warps 4 + q and 8 + q (the same TMEM lane quarter).
 
   if (warp < 4) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsLow));
@@ -418,8 +426,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         if (!(ok = mbar_wait(q_full, nq & 1, kStatusTimeoutMma))) break;
         ++nq;
         int s_left = 0;  // S products still to issue for this item
+        int last_j[2] = {-1, -1};  // last key step of each q tile (o_done[t] follows its P.V)
         for (int t = 0; t < 2; ++t)
-          for (int j = 0; j < it.j_count; ++j) s_left += tile_active(it, t, j) ? 1 : 0;
+          for (int j = 0; j < it.j_count; ++j)
+            if (tile_active(it, t, j)) {
+              ++s_left;
+              last_j[t] = j;
+            }
+        // A q tile without key steps in this item still completes its o_done.
+        auto finish_idle_tiles = [&]() {
+          for (int t = 0; t < 2; ++t)
+            if (last_j[t] < 0) mma_commit(&o_done[t]);
+        };
         auto slot_addr = [&](int idx) {
           return ring_addr + ((ubase + idx) % C::kSlots) * C::kTileBytes;
         };
@@ -478,6 +496,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               issue_pv_at(t, paddr(1, up(t, j)), first_pv[t]);
               first_pv[t] = false;
               ++n_act[t];
+              if (j == last_j[t]) mma_commit(&o_done[t]);
               prelease(1, up(t, j));
               if (tile_active(it, t, j + 1)) {
                 if (!(ok = pwait(0, up(t, j + 1)))) break;
@@ -487,7 +506,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             }
           }
           if (!ok) break;
-          mma_commit(o_done);
+          finish_idle_tiles();
           ubase += it.kc[0] + it.kc[1];
           continue;
         }
@@ -497,7 +516,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         };
 
         // Prologue: S(0) of both tiles (K_0's only readers, so its slot is
-        // released at once); the softmax takes tile A, then B.
+        // released at once).
         if (!(ok = wait_slot(0))) break;
         if (tile_active(it, 0, 0)) issue_s(0, 0);
         if (tile_active(it, 1, 0)) issue_s(1, 0);
@@ -511,6 +530,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               issue_pv(t, j, first_pv[t]);
               first_pv[t] = false;
               ++n_act[t];
+              if (j == last_j[t]) mma_commit(&o_done[t]);
             }
             if (j + 1 < it.j_count && tile_active(it, t, j + 1)) {
               if (!k_next_ready) {
@@ -529,7 +549,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (j + 1 < it.j_count) release(2 * (j + 1));
         }
         if (!ok) break;
-        mma_commit(o_done);
+        finish_idle_tiles();
         ubase += 2 * it.j_count;
       }
       // Drain: every MMA finished before TMEM can be released.
@@ -539,260 +559,251 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax / epilogue
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsHigh));
-    // Warps 4-7 take key columns [0, 64) of every S tile, warps 8-11 columns
-    // [64, 128).  Warps w and w + 4 read the same TMEM lane quarter (w & 3),
-    // i.e. the same 32 rows: partner threads own the two halves of one row
-    // and swap row values through `xchg` under named barrier 1 + quarter.
-    // All eight warps process tile A, then tile B, at every key step.
-    const int h = (warp - 4) / 4;            // column half
-    const int quarter = warp & 3;            // TMEM lane quarter of this warp
-    const int r = quarter * 32 + lane;       // row within a q tile
-    const int bar_id = 1 + quarter;
+    // Warpgroup t (warps 4-7: tile A, 8-11: tile B); thread = row r of its
+    // q tile, which is TMEM lane r (warp w reads lane quarter w % 4).
+    const int t = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
-    const int oc0 = min(64 * h, p.d_pad), oc1 = min(64 * h + 64, p.d_pad);  // O columns
+    const uint32_t s_tm = tmem + lane_base + t * 128;
+    const uint32_t o_tm = tmem + lane_base + 256 + t * 128;
     uint8_t* stage = stage_all + (warp - 4) * 4096;
-    // Swap `mine` with the partner's value; `okv` becomes the AND over the
-    // pair.  The first barrier guarantees the partner has read the previous
-    // value before it is overwritten; the fences order TMEM accesses of the
-    // two threads around the barriers.
-    auto exchange = [&](float mine, bool& okv) -> float {
-      tc_fence_before();
-      named_bar_sync(bar_id, 64);
-      xchg[h * kPfM + r] = mine;
-      okv = named_bar_and(bar_id, 64, okv);
-      tc_fence_after();
-      return xchg[(1 - h) * kPfM + r];
+    // O columns of this thread's row of tile u, col .. col + 15 (warp-collective).
+    auto load_o = [&](int u, int col, float (&v)[16]) {
+      uint32_t ov[16];
+      tmem_ld16(tmem + lane_base + 256 + u * 128 + col, ov);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(ov[e]);
     };
-    struct RowState {
-      int lo, hi;       // visible keys of this thread's row (hi < lo: none)
-      int act;          // key tiles consumed in this item
-      float m, l;       // running max (log2 domain) and this half's running sum
-    };
-    int n_act0 = 0, n_act1 = 0;  // S tiles consumed per q tile (s_full phases)
-    int n_done = 0;              // busy items finished (o_done phases)
-    int n_merge = 0;             // split tickets taken by this column half (part_done phases)
+    int n_s = 0;      // S tiles consumed (s_full[t] phases)
+    int n_busy = 0;   // busy items finished (o_done phases)
+    int n_merge = 0;  // split tickets taken by this warpgroup (part_done[t] phases)
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const PfItem it = prefill_item<kSplit>(p, ms, item);
-      RowState st[2];
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        st[t].lo = 0;
-        st[t].hi = -1;
-        st[t].act = 0;
-        st[t].m = -INFINITY;
-        st[t].l = 0.f;
-        if (r < it.tile[t].nrows) {
-          const long long grow = (long long)it.tile[t].row0 + r;  // row within the unit
-          const int qpos = p.kv_len - p.q_len + (int)(grow % p.q_len);
-          st[t].lo = first_key(ms, qpos);
-          st[t].hi = last_key(ms, qpos);
-        }
+      const TileInfo ti = t ? it.tile[1] : it.tile[0];
+      int lo = 0, hi = -1;  // visible keys of this row (hi < lo: none)
+      if (r < ti.nrows) {
+        const long long grow = (long long)ti.row0 + r;  // row within the unit
+        const int qpos = p.kv_len - p.q_len + (int)(grow % p.q_len);
+        lo = first_key(ms, qpos);
+        hi = last_key(ms, qpos);
       }
-      for (int j = 0; j < it.j_count && ok; ++j) {
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (!tile_active(it, t, j)) continue;
-          // One body for both tiles: the tile's state moves into `cs`.
-          RowState cs = t ? st[1] : st[0];
-          const KeyRange kr = t ? it.tile[1].kr : it.tile[0].kr;
-          const int nph = t ? n_act1 : n_act0;
-          const uint32_t s_tmem = tmem + lane_base + t * 128 + 64 * h;
-          const uint32_t o_tmem = tmem + lane_base + 256 + t * 128;
-          const int ktile0 = key_tile(it, t, j) * kPfN;
-          const int key0 = ktile0 + 64 * h;  // key of this half's column 0
-          const bool need_mask = !(ktile0 >= kr.all_lo && ktile0 + kPfN - 1 <= kr.all_hi);
-          const int clo = cs.lo - key0, chi = cs.hi - key0;  // visible columns
-          bool wok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], nph & 1, kStatusTimeoutSoftmax));
-          float x[64];
-          float mraw = -INFINITY;
-          bool small_y = false;
-          if (wok) {
-            tc_fence_after();
-            uint32_t s0[32], s1[32];
-            tmem_ld32(s_tmem + 0, s0);
-            tmem_ld32(s_tmem + 32, s1);
+      float m = -INFINITY;  // running max (log2 domain)
+      float l = 0.f;        // running sum
+      int act = 0;          // key tiles consumed in this item (the same in the whole warpgroup)
+      for (int j = 0; j < it.j_count; ++j) {
+        if (!tile_active(it, t, j)) continue;
+        const int ktile0 = key_tile(it, t, j) * kPfN;
+        const bool need_mask = !(ktile0 >= ti.kr.all_lo && ktile0 + kPfN - 1 <= ti.kr.all_hi);
+        ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], n_s & 1, kStatusTimeoutSoftmax));
+        ++n_s;
+        if (!ok) break;
+        tc_fence_after();
+        const int clo = lo - ktile0, chi = hi - ktile0;  // visible columns of this row
+        // Pass 1: the row's 128 scores, for its max (and, with a softcap, its
+        // min: when every |x / s| of the warp's rows is <= 1/2, tanh runs as
+        // an odd polynomial on the FMA pipe; the raw scores decide it).
+        bool small_y = false;
+        float mraw;
+        {
+          uint32_t sr[128];
+          tmem_ld128(s_tm, sr);
+          tmem_ld_wait();
+          auto xv = [&](int c) { return __uint_as_float(sr[c]); };
+          // Visible score, or -inf.
+          auto xm = [&](int c) { return c < clo || c > chi ? -INFINITY : xv(c); };
+          auto row_max = [&](auto score) {
+            float mx[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) mx[k] = fmaxf(score(2 * k), score(2 * k + 1));
+#pragma unroll
+            for (int c = 8; c < 128; c += 8)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) mx[k] = fmax3(mx[k], score(c + 2 * k), score(c + 2 * k + 1));
+            return fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+          };
+          if constexpr (kCap) {
+            float mx[4], mn[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              mx[k] = fmaxf(xv(2 * k), xv(2 * k + 1));
+              mn[k] = fminf(xv(2 * k), xv(2 * k + 1));
+            }
+#pragma unroll
+            for (int c = 8; c < 128; c += 8)
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                mx[k] = fmax3(mx[k], xv(c + 2 * k), xv(c + 2 * k + 1));
+                mn[k] = fmin3(mn[k], xv(c + 2 * k), xv(c + 2 * k + 1));
+              }
+            mraw = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
+            const float mna = fmin3(mn[0], mn[1], fminf(mn[2], mn[3]));
+            small_y = __all_sync(0xffffffffu, fmaxf(mraw, -mna) * p.cap_in <= 0.5f);
+            if (need_mask) mraw = row_max(xm);
+          } else {
+            mraw = need_mask ? row_max(xm) : row_max(xv);
+          }
+        }
+        const float mt = mraw == -INFINITY ? -INFINITY
+                         : kCap ? p.cap_out * tanh_fast(mraw * p.cap_in)
+                                : mraw * p.logit_scale;
+        // Rescale only when the max grew by more than 2^8 (or was -inf): the
+        // stale max keeps p <= 256, and O / l stays consistent.
+        const float m_new = fmaxf(m, mt);
+        const bool need =
+            (m_new > m + kRescaleThreshold) || (m == -INFINITY && m_new != -INFINITY);
+        const float alpha = need ? ex2(m - m_new) : 1.0f;  // 0 when m = -inf
+        if (need) {
+          l *= alpha;
+          m = m_new;
+        }
+        if (__any_sync(0xffffffffu, need) && act > 0) {
+          // This row of O_t (tcgen05.ld / st are warp-collective).
+          for (int c0 = 0; c0 < p.d_pad; c0 += 16) {
+            uint32_t ov[16];
+            tmem_ld16(o_tm + c0, ov);
             tmem_ld_wait();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-              x[c] = __uint_as_float(s0[c]);
-              x[32 + c] = __uint_as_float(s1[c]);
-            }
-            // Softcap: when every |x / s| of the warp's columns is <= 1/2 the
-            // tanh runs as a polynomial on the FMA pipe, leaving MUFU to ex2;
-            // the min of the raw scores (before masking) decides it.
-            if constexpr (kCap) {
-              float mx[8], mn[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) mx[i] = mn[i] = x[i];
-#pragma unroll
-              for (int c = 8; c < 64; ++c) {
-                mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-                mn[c & 7] = fminf(mn[c & 7], x[c]);
-              }
-              mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-              const float mnr = fminf(fminf(fminf(mn[0], mn[1]), fminf(mn[2], mn[3])),
-                                      fminf(fminf(mn[4], mn[5]), fminf(mn[6], mn[7])));
-              small_y = __all_sync(0xffffffffu, fmaxf(mraw, -mnr) * p.cap_in <= 0.5f);
-            }
-            if (!kCap || need_mask) {
-              // Row max of the raw scores over visible keys (8 chains); scale
-              // and softcap are increasing, so the log2-domain max is the
-              // transform of this one.
-              if (need_mask) {
-#pragma unroll
-                for (int c = 0; c < 64; ++c)
-                  if (c < clo || c > chi) x[c] = -INFINITY;
-              }
-              float mx[8];
-#pragma unroll
-              for (int i = 0; i < 8; ++i) mx[i] = x[i];
-#pragma unroll
-              for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-              mraw = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            }
+            for (int e = 0; e < 16; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st16(o_tm + c0, ov);
           }
-          const float mrow = fmaxf(mraw, exchange(mraw, wok));
-          if (!wok) {
-            ok = false;
-            break;
-          }
-          // The same transform of the same value in both halves: the row's
-          // max is bitwise equal in the two partner threads.
-          const float mt = mrow == -INFINITY ? -INFINITY
-                           : kCap ? p.cap_out * tanh_fast(mrow * p.cap_in)
-                                  : mrow * p.logit_scale;
-          // Rescale only when the max grew by more than 2^8 (or was -inf):
-          // the stale max keeps p <= 256, and O / l stays consistent.
-          const float m_new = fmaxf(cs.m, mt);
-          const bool need =
-              (m_new > cs.m + kRescaleThreshold) || (cs.m == -INFINITY && m_new != -INFINITY);
-          const float alpha = need ? ex2(cs.m - m_new) : 1.0f;  // 0 when m = -inf
-          if (need) {
-            cs.l *= alpha;
-            cs.m = m_new;
-          }
-          if (__any_sync(0xffffffffu, need) && cs.act > 0) {
-            // This half's O columns; tcgen05.ld/st are warp-collective.
-            for (int c0 = oc0; c0 < oc1; c0 += 16) {
-              uint32_t ov[16];
-              tmem_ld16(o_tmem + c0, ov);
-              tmem_ld_wait();
-#pragma unroll
-              for (int e = 0; e < 16; ++e)
-                ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-              tmem_st16(o_tmem + c0, ov);
-            }
-            tmem_st_wait();
-          }
-          const float base = cs.m == -INFINITY ? 0.f : cs.m;
-          float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-          // p = 2^(logit - base) as bf16 pairs into TMEM over S: the 32 keys of
-          // chunk g of the tile land in columns [16g, 16g + 16).  Both halves
-          // loaded their S before the exchange, so no unread score is
-          // overwritten.  A hidden key (x = -inf) gives p = 0.
-          const uint32_t p_tmem = tmem + lane_base + t * 128 + 32 * h;
-          auto emit = [&](auto logit, auto zero_hidden) {
-#pragma unroll
-            for (int q2 = 0; q2 < 2; ++q2) {
-              uint32_t pk[16];
-#pragma unroll
-              for (int c = 0; c < 16; ++c) {
-                float pe[2];
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                  const int col = 32 * q2 + 2 * c + e;
-                  pe[e] = ex2(logit(x[col]));
-                  if (zero_hidden(col)) pe[e] = 0.f;
-                }
-                ls[c & 7] += pe[0] + pe[1];
-                pk[c] = pack_bf16(pe[0], pe[1]);
-              }
-              tmem_st16(p_tmem + 16 * q2, pk);
-            }
-          };
-          auto none = [](int) { return false; };
-          if constexpr (!kCap) {
-            const float sc = p.logit_scale;
-            emit([&](float v) { return fmaf(v, sc, -base); }, none);
-          } else {
-            // With a softcap a hidden key's logit is not -inf, so its p is
-            // zeroed explicitly.
-            auto hidden = [&](int col) { return x[col] == -INFINITY; };
-            if (small_y) {
-              // The odd tanh polynomial with cap_in^(2k+1) * cap_out folded
-              // in: cap_out * tanh(x * cap_in) = x * Q(x^2).
-              const float ci2 = p.cap_in * p.cap_in, cc = p.cap_out * p.cap_in;
-              if constexpr (kCapDeg == 5) {
-                const float q0 = cc * kTanh5C1, q1 = cc * ci2 * kTanh5C3;
-                const float q2c = cc * ci2 * ci2 * kTanh5C5;
-                auto logit = [&](float v) {
-                  const float v2 = v * v;
-                  return fmaf(v, fmaf(fmaf(q2c, v2, q1), v2, q0), -base);
-                };
-                if (need_mask) emit(logit, hidden);
-                else emit(logit, none);
-              } else {
-                const float q0 = cc * kTanhC1, q1 = cc * ci2 * kTanhC3;
-                const float q2c = cc * ci2 * ci2 * kTanhC5, q3 = cc * ci2 * ci2 * ci2 * kTanhC7;
-                auto logit = [&](float v) {
-                  const float v2 = v * v;
-                  return fmaf(v, fmaf(fmaf(fmaf(q3, v2, q2c), v2, q1), v2, q0), -base);
-                };
-                if (need_mask) emit(logit, hidden);
-                else emit(logit, none);
-              }
-            } else {
-              const float co = p.cap_out, ci = p.cap_in;
-              auto logit = [&](float v) { return fmaf(co, tanh_fast(v * ci), -base); };
-              if (need_mask) emit(logit, hidden);
-              else emit(logit, none);
-            }
-          }
-          cs.l += ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
           tmem_st_wait();
-          tc_fence_before();
-          mbar_arrive(&p_full[t]);
-          ++cs.act;
-          if (t) {
-            st[1] = cs;
-            ++n_act1;
-          } else {
-            st[0] = cs;
-            ++n_act0;
-          }
         }
-      }
-      if (!ok) break;
-      // ---- epilogue: o = O / l as bf16.  The next item's first P.V may
-      // overwrite O only after the next P arrival of all eight warps, which
-      // follows these (waited) TMEM loads in program order.  One barrier
-      // covers both tiles: every MMA of the item has finished.
-      bool eok = true;
-      if (it.busy) {
-        eok = __all_sync(0xffffffffu, mbar_wait(o_done, n_done & 1, kStatusTimeoutEpilogue));
-        ++n_done;
-      }
-      // Row sums: the two halves add the same two values in the same order.
-      float lsum[2];
+        const float base = m == -INFINITY ? 0.f : m;
+        // Pass 2: p = 2^(logit - base) as bf16 pairs into TMEM over S, 32
+        // keys at a time: the scores of keys 32g .. 32g + 31 are read again
+        // (the next group's read is in flight while this one is computed) and
+        // their P lands in columns [16g, 16g + 16), all of whose scores were
+        // read before.  Pairs [kEmuFrom, 16) of each group take the FMA-pipe
+        // 2^x on tiles without a mask; a hidden key gives p = 0 (its logit is
+        // -inf, or it is zeroed explicitly).
+        f2 acc[4] = {0ull, 0ull, 0ull, 0ull};
+        auto emit = [&](auto logit2, auto emu, auto hidden) {
+          uint32_t buf[2][32];
+          tmem_ld32(s_tm, buf[0]);
+          tmem_ld_wait();
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const float other = exchange(st[t].l, eok);
-        lsum[t] = h == 0 ? st[t].l + other : other + st[t].l;
+          for (int g = 0; g < 4; ++g) {
+            if (g < 3) tmem_ld32(s_tm + 32 * (g + 1), buf[(g + 1) & 1]);
+            const uint32_t(&sv)[32] = buf[g & 1];
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              float xa = __uint_as_float(sv[2 * c]), xb = __uint_as_float(sv[2 * c + 1]);
+              const int col = 32 * g + 2 * c;
+              bool ha = false, hb = false;
+              if constexpr (decltype(hidden)::value) {
+                ha = col < clo || col > chi;
+                hb = col + 1 < clo || col + 1 > chi;
+                if constexpr (!kCap) {  // -inf logits give p = 0 by themselves
+                  if (ha) xa = -INFINITY;
+                  if (hb) xb = -INFINITY;
+                }
+              }
+              const f2 y = logit2(f2_pack(xa, xb));
+              f2 pv = (decltype(emu)::value && c >= kEmuFrom) ? exp2_poly_x2(y) : exp2_mufu_x2(y);
+              if constexpr (decltype(hidden)::value && kCap) {
+                float a, b;
+                f2_unpack(pv, a, b);
+                pv = f2_pack(ha ? 0.f : a, hb ? 0.f : b);
+              }
+              acc[c & 3] = f2_add(acc[c & 3], pv);
+              pk[c] = pack_bf16_f2(pv);
+            }
+            tmem_st16(s_tm + 16 * g, pk);
+            if (g < 3) tmem_ld_wait();
+          }
+        };
+        using Yes = std::true_type;
+        using No = std::false_type;
+        const f2 nb = f2_pack(-base, -base);
+        if constexpr (!kCap) {
+          const f2 sc = f2_pack(p.logit_scale, p.logit_scale);
+          auto logit = [&](f2 v) { return f2_fma(v, sc, nb); };
+          if (need_mask) emit(logit, No(), Yes());
+          else emit(logit, Yes(), No());
+        } else if (small_y) {
+          // cap_out * tanh(x * cap_in) = x * Q(x^2), the odd polynomial with
+          // cap_in^(2k+1) * cap_out folded into its coefficients.
+          const float ci2 = p.cap_in * p.cap_in, cc = p.cap_out * p.cap_in;
+          if constexpr (kCapDeg == 5) {
+            const f2 q0 = f2_pack(cc * kTanh5C1, cc * kTanh5C1);
+            const f2 q1 = f2_pack(cc * ci2 * kTanh5C3, cc * ci2 * kTanh5C3);
+            const f2 q2 = f2_pack(cc * ci2 * ci2 * kTanh5C5, cc * ci2 * ci2 * kTanh5C5);
+            auto logit = [&](f2 v) {
+              const f2 v2 = f2_mul(v, v);
+              return f2_fma(v, f2_fma(f2_fma(q2, v2, q1), v2, q0), nb);
+            };
+            if (need_mask) emit(logit, No(), Yes());
+            else emit(logit, Yes(), No());
+          } else {
+            const f2 q0 = f2_pack(cc * kTanhC1, cc * kTanhC1);
+            const f2 q1 = f2_pack(cc * ci2 * kTanhC3, cc * ci2 * kTanhC3);
+            const f2 q2 = f2_pack(cc * ci2 * ci2 * kTanhC5, cc * ci2 * ci2 * kTanhC5);
+            const f2 q3 = f2_pack(cc * ci2 * ci2 * ci2 * kTanhC7, cc * ci2 * ci2 * ci2 * kTanhC7);
+            auto logit = [&](f2 v) {
+              const f2 v2 = f2_mul(v, v);
+              return f2_fma(v, f2_fma(f2_fma(f2_fma(q3, v2, q2), v2, q1), v2, q0), nb);
+            };
+            if (need_mask) emit(logit, No(), Yes());
+            else emit(logit, Yes(), No());
+          }
+        } else {
+          // Large arguments (rare): the hardware tanh, every exponential on MUFU.
+          const float co = p.cap_out, ci = p.cap_in;
+          auto logit = [&](f2 v) {
+            float a, b;
+            f2_unpack(v, a, b);
+            return f2_pack(fmaf(co, tanh_fast(a * ci), -base), fmaf(co, tanh_fast(b * ci), -base));
+          };
+          if (need_mask) emit(logit, No(), Yes());
+          else emit(logit, No(), No());
+        }
+        {
+          float a0, a1, b0, b1, c0, c1, d0, d1;
+          f2_unpack(acc[0], a0, a1);
+          f2_unpack(acc[1], b0, b1);
+          f2_unpack(acc[2], c0, c1);
+          f2_unpack(acc[3], d0, d1);
+          l += ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&p_full[t]);
+        ++act;
       }
-      if (!eok) break;
+      // Paired items (every item of a launch, or none): the two warpgroups
+      // meet at a named barrier below, so a warpgroup that gave up on a wait
+      // still goes there (with ok = false) instead of leaving at once.
+      const bool pair_x = kSplit && it.paired;
+      if (!ok && !pair_x) break;
+      // ---- epilogue.  The next item's first P.V of this tile may overwrite
+      // O only after this warpgroup's next P arrival, which follows these
+      // (waited) TMEM loads in program order.
+      if (it.busy) {
+        const uint32_t ph = n_busy & 1;
+        ++n_busy;
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_done[t], ph, kStatusTimeoutEpilogue));
+        // Paired items: this warpgroup also reads the other tile's O.
+        if (ok && pair_x)
+          ok = __all_sync(0xffffffffu, mbar_wait(&o_done[1 - t], ph, kStatusTimeoutEpilogue));
+        if (!ok && !pair_x) break;
+      }
       tc_fence_after();
-      // Write this warp's 32 rows, columns [oc0, oc1), as bf16 through its
+      // Write this warp's 32 rows, columns [c0, c0 + 64), as bf16 through its
       // 128B-swizzled 32-row staging box and one TMA store (rows past the
       // unit's end are not written).  value16(col, v) fills v with the fp32
       // outputs of columns col .. col + 15.
-      auto store_rows = [&](const TileInfo& ti, auto value16) {
+      auto store_box = [&](const TileInfo& tile, int c0, auto value16) {
         if (lane == 0) bulk_wait_read();  // the previous store has read the box
         __syncwarp();
-        for (int c1 = 0; c1 < oc1 - oc0; c1 += 16) {
+        const int cw = min(64, p.d_pad - c0);
+        for (int c1 = 0; c1 < cw; c1 += 16) {
           float v[16];
-          value16(oc0 + c1, v);
+          value16(c0 + c1, v);
 #pragma unroll
           for (int g = 0; g < 2; ++g) {  // 8 columns = one 16-byte chunk
             const uint4 w = make_uint4(pack_bf16(v[8 * g], v[8 * g + 1]),
@@ -805,88 +816,97 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) {
-          tma_store_3d(&tm_o, stage, oc0, ti.row0 + quarter * 32, it.unit);
+          tma_store_3d(&tm_o, stage, c0, tile.row0 + quarter * 32, it.unit);
           bulk_commit();
         }
       };
-      // O columns col .. col + 15 of this thread's row of tile t from TMEM
-      // (warp-collective).
-      auto load_o = [&](int t, int col, float (&v)[16]) {
-        uint32_t ov[16];
-        tmem_ld16(tmem + lane_base + 256 + t * 128 + col, ov);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) v[e] = __uint_as_float(ov[e]);
-      };
       if constexpr (!kSplit) {
-        for (int t = 0; t < 2; ++t) {
-          const TileInfo ti = t ? it.tile[1] : it.tile[0];
-          if (ti.nrows <= 0 || quarter * 32 >= ti.nrows || oc0 >= oc1) continue;
-          const bool have = (t ? st[1].act : st[0].act) > 0;
-          const float L = t ? lsum[1] : lsum[0];
-          const bool live = have && L > 0.f;
-          const float inv = live ? 1.0f / L : 0.f;
-          store_rows(ti, [&](int col, float (&v)[16]) {
-            if (have) {
-              load_o(t, col, v);
+        if (ti.nrows > 0 && quarter * 32 < ti.nrows) {
+          const bool have = act > 0;  // warp-uniform
+          const bool live = have && l > 0.f;
+          const float inv = live ? 1.0f / l : 0.f;
+          for (int c0 = 0; c0 < p.d_pad; c0 += 64)
+            store_box(ti, c0, [&](int col, float (&v)[16]) {
+              if (have) {
+                load_o(t, col, v);
 #pragma unroll
-              for (int e = 0; e < 16; ++e) v[e] = live ? v[e] * inv : 0.f;
-            } else {
+                for (int e = 0; e < 16; ++e) v[e] = live ? v[e] * inv : 0.f;
+              } else {
 #pragma unroll
-              for (int e = 0; e < 16; ++e) v[e] = 0.f;
-            }
-          });
+                for (int e = 0; e < 16; ++e) v[e] = 0.f;
+              }
+            });
         }
       } else {
         // ---- key splits.  Each split leaves a partial per row: O
-        // (unnormalised, fp32), m and l, with m and l kept per column half so
-        // each half's merge reads only what its own warps wrote.  A paired
-        // item holds two splits of the same rows (tiles A and B), combined
-        // here first, so a row group has splits / 2 partials.  The four
-        // warps of a column half take one ticket per row group; in the CTA
-        // that brings the last partial they merge all of them, in partial
-        // order (deterministic), sharing the rows and columns between them.
-        const int np = it.paired ? p.splits / 2 : p.splits;
-        const int psplit = it.paired ? it.split / 2 : it.split;
-        for (int t = 0; t < (it.paired ? 1 : 2); ++t) {
-          const TileInfo ti = t ? it.tile[1] : it.tile[0];
-          if (ti.nrows <= 0) continue;  // the same for every warp
-          const int ptile = it.paired ? it.pair_index : it.pair_index * 2 + t;
+        // (unnormalised, fp32), m and l.  Unpaired items: warpgroup t writes
+        // the partial of its own q tile, all columns.  Paired items (tiles A
+        // and B are two splits of the same rows): the two warpgroups swap
+        // their rows' (m, l), combine both tiles' O into one partial, and
+        // each writes columns [64t, 64t + 64) of it.  One ticket per (row
+        // tile, warpgroup); in the CTA that brings the last partial, the four
+        // warps of the warpgroup merge all of them in partial order
+        // (deterministic), sharing the rows and columns between them.
+        const bool paired = it.paired;
+        float mo = -INFINITY, lo_ = 0.f;  // the other tile's (m, l) (paired)
+        if (paired) {
+          // Warps 4 + q and 8 + q hold the same rows.  The first barrier
+          // keeps this write behind the partner's read of the previous
+          // item's value; the second publishes it and ANDs the two ok flags.
+          tc_fence_before();
+          named_bar_sync(1 + quarter, 64);
+          xchg[t * kPfM + r] = make_float2(m, l);
+          ok = named_bar_and(1 + quarter, 64, ok);
+          tc_fence_after();
+          const float2 other = xchg[(1 - t) * kPfM + r];
+          mo = other.x;
+          lo_ = other.y;
+          if (!ok) break;
+        }
+        const TileInfo& rt = it.tile[0];  // the row tile of a paired item
+        const TileInfo& wt = paired ? rt : ti;
+        const int cw0 = paired ? min(64 * t, p.d_pad) : 0;
+        const int cw1 = paired ? min(64 * t + 64, p.d_pad) : p.d_pad;
+        const int hh = paired ? t : 0;  // (m, l) and ticket slot
+        const int np = paired ? p.splits / 2 : p.splits;
+        const int psplit = paired ? it.split / 2 : it.split;
+        if (wt.nrows > 0) {  // the same for every warp of the warpgroup
+          const int ptile = paired ? it.pair_index : it.pair_index * 2 + t;
           const long long blk = (long long)ptile * np;
           auto po_of = [&](int sp) {
             return reinterpret_cast<float4*>(p.ws_o + (blk + sp) * (long long)p.d_pad * kPfM);
           };
-          auto ml_of = [&](int sp) { return p.ws_ml + ((blk + sp) * 2 + h) * 2 * kPfM; };
-          // Cluster merge: the combined partial stays in this CTA's shared
-          // memory (the K/V ring and staging area are idle after the CTA's
-          // only item): O as fp32 rows of d_pad + 4 floats, m and l per row.
-          const bool to_smem = it.paired && p.cluster_merge > 0;
-          if (quarter * 32 < ti.nrows && oc0 < oc1) {
-            // This row's tiles: t alone, or A and B rescaled to their common
-            // max.  A tile whose rows saw no key (act = 0, or m = -inf) adds
-            // nothing; an empty partial has m = -inf, l = 0 and O = 0.
-            const RowState& sa = t ? st[1] : st[0];
-            const bool use_b = it.paired;
-            const bool ha = sa.act > 0 && sa.m != -INFINITY;
-            const bool hb = use_b && st[1].act > 0 && st[1].m != -INFINITY;
-            float m = ha ? sa.m : -INFINITY;
-            if (hb) m = fmaxf(m, st[1].m);
-            const float wa = ha ? ex2(sa.m - m) : 0.f;
-            const float wb = hb ? ex2(st[1].m - m) : 0.f;
-            const float L = wa * (t ? lsum[1] : lsum[0]) + (use_b ? wb * lsum[1] : 0.f);
+          auto ml_of = [&](int sp) { return p.ws_ml + ((blk + sp) * 2 + hh) * 2 * kPfM; };
+          // Cluster merge: the partial stays in this CTA's shared memory (the
+          // K/V ring and staging area are idle after the CTA's only item): O
+          // as fp32 rows of d_pad + 4 floats, m and l per row.
+          const bool to_smem = paired && p.cluster_merge > 0;
+          if (quarter * 32 < wt.nrows && cw0 < cw1) {
+            // Tile A = this warpgroup's (paired: t = 0) or the only tile.
+            const int act_a = paired ? it.kc[0] : act, act_b = paired ? it.kc[1] : 0;
+            const float ma = paired ? (t ? mo : m) : m, la = paired ? (t ? lo_ : l) : l;
+            const float mb = paired ? (t ? m : mo) : -INFINITY, lb = paired ? (t ? l : lo_) : 0.f;
+            const bool ha = act_a > 0 && ma != -INFINITY;
+            const bool hb = act_b > 0 && mb != -INFINITY;
+            float mc = ha ? ma : -INFINITY;
+            if (hb) mc = fmaxf(mc, mb);
+            const float wa = ha ? ex2(ma - mc) : 0.f;
+            const float wb = hb ? ex2(mb - mc) : 0.f;
+            const float L = wa * la + (hb ? wb * lb : 0.f);
+            const int ua = paired ? 0 : t;  // TMEM O of tile A
             float4* po = po_of(psplit);
             float* crow = reinterpret_cast<float*>(ring) + r * (p.d_pad + 4);
-            for (int c0 = oc0; c0 < oc1; c0 += 16) {
+            for (int c0 = cw0; c0 < cw1; c0 += 16) {
               float v[16];
 #pragma unroll
               for (int e = 0; e < 16; ++e) v[e] = 0.f;
-              if (sa.act > 0) {  // warp-uniform
+              if (act_a > 0) {  // warp-uniform
                 float a[16];
-                load_o(t, c0, a);
+                load_o(ua, c0, a);
 #pragma unroll
                 for (int e = 0; e < 16; ++e) v[e] = wa * a[e];
               }
-              if (use_b && st[1].act > 0) {
+              if (act_b > 0) {
                 float b[16];
                 load_o(1, c0, b);
 #pragma unroll
@@ -902,113 +922,119 @@ __global__ void __launch_bounds__(kPfThreads, 1)
               }
             }
             float* pml = to_smem ? reinterpret_cast<float*>(stage_all) : ml_of(psplit);
-            if (!to_smem || h == 0) {
-              pml[r] = ha || hb ? m : -INFINITY;
+            if (!to_smem || t == 0) {
+              pml[r] = ha || hb ? mc : -INFINITY;
               pml[kPfM + r] = L;
             }
           }
-          if (to_smem) continue;  // merged after the cluster barrier
-          // The ticket: every thread's partial is visible device-wide before
-          // one thread of the half counts it (bounded waits: a warp that gave
-          // up elsewhere makes the others give up here, not hang).
-          __threadfence();
-          mbar_arrive(&part_done[h]);
-          const uint32_t mph = n_merge & 1;
-          ++n_merge;
-          unsigned int* tk = p.tickets + ptile * 2 + h;
-          if (quarter == 0 && lane == 0) {
-            int f = -1;
-            if (mbar_wait(&part_done[h], mph, kStatusTimeoutEpilogue))
-              f = atomicAdd(tk, 1u) == (unsigned)(np - 1) ? 1 : 0;
-            merge_flag[h] = f;
-            mbar_arrive(&flag_ready[h]);
-          }
-          const int flag = __all_sync(0xffffffffu, mbar_wait(&flag_ready[h], mph, kStatusTimeoutEpilogue))
-                               ? *(volatile int*)&merge_flag[h]
-                               : -1;
-          if (flag < 0) {
-            ok = false;
-            break;
-          }
-          const bool last = flag == 1;
-          if (!last) continue;
-          __threadfence();
-          if (quarter == 0 && lane == 0) atomicExch(tk, 0u);  // ready for the next call
-          // Work of this warp: row group rg (32 rows), column part `part`
-          // of this half (whole 16-column chunks).  Fewer than three row
-          // groups: the idle warps take column parts instead.
-          const int nq = (ti.nrows + 31) / 32;
-          const int parts = nq == 1 ? 4 : nq == 2 ? 2 : 1;
-          const int rg = parts == 1 ? quarter : quarter % nq;
-          const int part = parts == 1 ? 0 : quarter / nq;
-          const int nch = (oc1 - oc0) / 16;
-          const int cb = oc0 + 16 * (nch * part / parts);
-          const int ce = oc0 + 16 * (nch * (part + 1) / parts);
-          if (rg >= nq || cb >= ce) continue;
-          const int row = rg * 32 + lane;  // < 128: partial rows past nrows exist
-          // Row max and row sum over the partials in one pass, eight (m, l)
-          // loads in flight at a time; the sum is rescaled when a later batch
-          // raises the max.
-          float M = -INFINITY, Ls = 0.f;
-          for (int sp0 = 0; sp0 < np; sp0 += 8) {
-            float mv[8], lv[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const bool in = sp0 + i < np;
-              mv[i] = in ? __ldcg(ml_of(sp0 + i) + row) : -INFINITY;
-              lv[i] = in ? __ldcg(ml_of(sp0 + i) + kPfM + row) : 0.f;
+          if (!to_smem) {
+            // The ticket: every thread's partial is visible device-wide before
+            // one thread of the warpgroup counts it (bounded waits: a warp that
+            // gave up elsewhere makes the others give up here, not hang).
+            __threadfence();
+            mbar_arrive(&part_done[t]);
+            const uint32_t mph = n_merge & 1;
+            ++n_merge;
+            unsigned int* tk = p.tickets + ptile * 2 + hh;
+            if (quarter == 0 && lane == 0) {
+              int f = -1;
+              if (mbar_wait(&part_done[t], mph, kStatusTimeoutEpilogue))
+                f = atomicAdd(tk, 1u) == (unsigned)(np - 1) ? 1 : 0;
+              merge_flag[t] = f;
+              mbar_arrive(&flag_ready[t]);
             }
-            float mb = M;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mb = fmaxf(mb, mv[i]);
-            if (mb != -INFINITY) {
-              if (M != -INFINITY) Ls *= ex2(M - mb);
-#pragma unroll
-              for (int i = 0; i < 8; ++i) Ls += mv[i] == -INFINITY ? 0.f : ex2(mv[i] - mb) * lv[i];
-              M = mb;
+            const int flag =
+                __all_sync(0xffffffffu, mbar_wait(&flag_ready[t], mph, kStatusTimeoutEpilogue))
+                    ? *(volatile int*)&merge_flag[t]
+                    : -1;
+            if (flag < 0) {
+              ok = false;
+              break;
             }
-          }
-          const float inv = Ls > 0.f ? 1.0f / Ls : 0.f;
-          __nv_bfloat16* orow = p.o + ((long long)it.unit * p.rows + ti.row0 + row) * p.head_dim;
-          for (int col = cb; col < ce; col += 16) {
-            float v[16];
+            if (flag == 1) {
+              __threadfence();
+              if (quarter == 0 && lane == 0) atomicExch(tk, 0u);  // ready for the next call
+              // Work of this warp: row group rg (32 rows), column part `part`
+              // of [cw0, cw1) (whole 16-column chunks).  Fewer than three row
+              // groups: the idle warps take column parts instead.
+              const int nq = (wt.nrows + 31) / 32;
+              const int parts = nq == 1 ? 4 : nq == 2 ? 2 : 1;
+              const int rg = parts == 1 ? quarter : quarter % nq;
+              const int part = parts == 1 ? 0 : quarter / nq;
+              const int nch = (cw1 - cw0) / 16;
+              const int cb = cw0 + 16 * (nch * part / parts);
+              const int ce = cw0 + 16 * (nch * (part + 1) / parts);
+              if (rg < nq && cb < ce) {
+                const int row = rg * 32 + lane;  // < 128: partial rows past nrows exist
+                // Row max and row sum over the partials in one pass, eight
+                // (m, l) loads in flight at a time; the sum is rescaled when a
+                // later batch raises the max.
+                float M = -INFINITY, Ls = 0.f;
+                for (int sp0 = 0; sp0 < np; sp0 += 8) {
+                  float mv[8], lv[8];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = 0.f;
-            // Eight partials per batch: their m and O loads all in flight
-            // together (past the last partial the loads read partial 0 with
-            // weight 0).
-            for (int sp0 = 0; sp0 < np; sp0 += 8) {
-              float mv[8];
-              float x8[8][16];
+                  for (int i = 0; i < 8; ++i) {
+                    const bool in = sp0 + i < np;
+                    mv[i] = in ? __ldcg(ml_of(sp0 + i) + row) : -INFINITY;
+                    lv[i] = in ? __ldcg(ml_of(sp0 + i) + kPfM + row) : 0.f;
+                  }
+                  float mb8 = M;
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const int sp = sp0 + i < np ? sp0 + i : 0;
-                mv[i] = sp0 + i < np ? __ldcg(ml_of(sp) + row) : -INFINITY;
-                const float4* src = po_of(sp) + row;
+                  for (int i = 0; i < 8; ++i) mb8 = fmaxf(mb8, mv[i]);
+                  if (mb8 != -INFINITY) {
+                    if (M != -INFINITY) Ls *= ex2(M - mb8);
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                  const float4 f = __ldcg(src + (col / 4 + g) * kPfM);
-                  x8[i][4 * g] = f.x;
-                  x8[i][4 * g + 1] = f.y;
-                  x8[i][4 * g + 2] = f.z;
-                  x8[i][4 * g + 3] = f.w;
+                    for (int i = 0; i < 8; ++i)
+                      Ls += mv[i] == -INFINITY ? 0.f : ex2(mv[i] - mb8) * lv[i];
+                    M = mb8;
+                  }
+                }
+                const float inv = Ls > 0.f ? 1.0f / Ls : 0.f;
+                __nv_bfloat16* orow =
+                    p.o + ((long long)it.unit * p.rows + wt.row0 + row) * p.head_dim;
+                for (int col = cb; col < ce; col += 16) {
+                  float v[16];
+#pragma unroll
+                  for (int e = 0; e < 16; ++e) v[e] = 0.f;
+                  // Eight partials per batch: their m and O loads all in
+                  // flight together (past the last partial the loads read
+                  // partial 0 with weight 0).
+                  for (int sp0 = 0; sp0 < np; sp0 += 8) {
+                    float mv[8];
+                    float x8[8][16];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                      const int sp = sp0 + i < np ? sp0 + i : 0;
+                      mv[i] = sp0 + i < np ? __ldcg(ml_of(sp) + row) : -INFINITY;
+                      const float4* src = po_of(sp) + row;
+#pragma unroll
+                      for (int g = 0; g < 4; ++g) {
+                        const float4 f = __ldcg(src + (col / 4 + g) * kPfM);
+                        x8[i][4 * g] = f.x;
+                        x8[i][4 * g + 1] = f.y;
+                        x8[i][4 * g + 2] = f.z;
+                        x8[i][4 * g + 3] = f.w;
+                      }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                      const float w = mv[i] == -INFINITY ? 0.f : ex2(mv[i] - M) * inv;
+#pragma unroll
+                      for (int e = 0; e < 16; ++e) v[e] = fmaf(w, x8[i][e], v[e]);
+                    }
+                  }
+                  if (row < wt.nrows) {
+                    // 8 columns (16 bytes) at a time; head_dim is a multiple of 8.
+#pragma unroll
+                    for (int g = 0; g < 2; ++g)
+                      if (col + 8 * g < p.head_dim)
+                        *reinterpret_cast<uint4*>(orow + col + 8 * g) = make_uint4(
+                            pack_bf16(v[8 * g], v[8 * g + 1]), pack_bf16(v[8 * g + 2], v[8 * g + 3]),
+                            pack_bf16(v[8 * g + 4], v[8 * g + 5]),
+                            pack_bf16(v[8 * g + 6], v[8 * g + 7]));
+                  }
                 }
               }
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const float w = mv[i] == -INFINITY ? 0.f : ex2(mv[i] - M) * inv;
-#pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = fmaf(w, x8[i][e], v[e]);
-              }
-            }
-            if (row < ti.nrows) {
-              // 8 columns (16 bytes) at a time; head_dim is a multiple of 8.
-#pragma unroll
-              for (int g = 0; g < 2; ++g)
-                if (col + 8 * g < p.head_dim)
-                  *reinterpret_cast<uint4*>(orow + col + 8 * g) =
-                      make_uint4(pack_bf16(v[8 * g], v[8 * g + 1]), pack_bf16(v[8 * g + 2], v[8 * g + 3]),
-                                 pack_bf16(v[8 * g + 4], v[8 * g + 5]), pack_bf16(v[8 * g + 6], v[8 * g + 7]));
             }
           }
         }

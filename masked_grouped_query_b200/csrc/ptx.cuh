@@ -257,6 +257,13 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr));
 }
+// 32 lanes x 128 columns (the whole of a 128-column S tile's rows), straight
+// into r; the registers are valid only after tmem_ld_wait().
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, uint32_t (&r)[128]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    tmem_ld32(taddr + 32 * q, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * q]));
+}
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -366,6 +373,103 @@ __device__ __forceinline__ float tanh_poly_small(float y) {
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Three-input max / min (sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// ---------------------------------------------------------------- fp32 pairs
+// sm_100 executes add / mul / fma on two fp32 values held in a 64-bit
+// register pair with one instruction.  f2 is such a pair (lo, hi).
+typedef uint64_t f2;
+__device__ __forceinline__ f2 f2_pack(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(f2 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f2 f2_fma(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ f2 f2_add(f2 a, f2 b) {
+  f2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 f2_sub(f2 a, f2 b) {
+  f2 d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ f2 f2_mul(f2 a, f2 b) {
+  f2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// a + b rounded toward -infinity.
+__device__ __forceinline__ f2 f2_add_rm(f2 a, f2 b) {
+  f2 d;
+  asm("add.rm.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// 2^f for f in [0, 1]: the cubic of least maximum relative error (7.5e-5),
+// fitted by fit_exp2_poly.py next to this file.
+constexpr float kExp2C0 = 0.9999251961708069f;
+constexpr float kExp2C1 = 0.6958335638046265f;
+constexpr float kExp2C2 = 0.22606714069843292f;
+constexpr float kExp2C3 = 0.07802452892065048f;
+
+// 2^y for a pair of y <= 2^7 without the MUFU unit (Cody-Waite): y is
+// clamped to >= -126, split as y = j + f with j = floor(y) (the add of
+// 1.5 * 2^23 rounded toward -inf leaves j in the low mantissa bits of the
+// sum) and f in [0, 1); the result is P(f) with j added to its exponent
+// field, which the clamp keeps >= 0.  Relative error 7.5e-5 for y >= -125;
+// below that the result is a non-negative value under 2^-124, not exactly
+// 2^y (callers use it only where such values are negligible next to the
+// row's largest term, 2^0 or more).
+__device__ __forceinline__ f2 exp2_poly_x2(f2 y) {
+  float a, b;
+  f2_unpack(y, a, b);
+  const f2 yc = f2_pack(fmaxf(a, -126.f), fmaxf(b, -126.f));
+  const f2 magic = f2_pack(12582912.f, 12582912.f);
+  const f2 t = f2_add_rm(yc, magic);
+  const f2 fr = f2_sub(yc, f2_sub(t, magic));
+  f2 q = f2_fma(fr, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
+  q = f2_fma(q, fr, f2_pack(kExp2C1, kExp2C1));
+  q = f2_fma(q, fr, f2_pack(kExp2C0, kExp2C0));
+  uint32_t t0, t1, q0, q1;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(q0), "=r"(q1) : "l"(q));
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(q0 + (t0 << 23)), "r"(q1 + (t1 << 23)));
+  return r;
+}
+
+// Two hardware ex2 (MUFU) on a pair.
+__device__ __forceinline__ f2 exp2_mufu_x2(f2 y) {
+  float a, b;
+  f2_unpack(y, a, b);
+  return f2_pack(ex2(a), ex2(b));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16_f2(f2 v) {
+  float a, b;
+  f2_unpack(v, a, b);
+  return pack_bf16(a, b);
 }
 
 }  // namespace gqa
