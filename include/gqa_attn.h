@@ -87,14 +87,21 @@ extern "C" {
  * The call validates, plans and enqueues 1 kernel (a memset when kv_len == 0,
  * nothing when o is empty) on `stream` and returns without synchronising.
  * Key-split partials live in a library-owned workspace per (device, stream),
- * allocated with cudaMalloc on first need and grown on demand (so the first
- * call of a new size synchronises the device); calls on one stream are
- * ordered, calls on different streams do not share workspace.  Partials of
- * the split-KV decode kernel and of the tcgen05 kernel's key splits use it;
- * when every (batch, kv head) has one 128-row tile and its CTAs fit on the
- * device at once, the tcgen05 kernel is launched as one thread-block cluster
- * per (batch, kv head) and merges its partials in distributed shared memory
- * instead.
+ * allocated with cudaMalloc on first need; calls on one stream are ordered,
+ * calls on different streams do not share workspace.  A call that needs more
+ * than the stream's workspace allocates a bigger one (no synchronisation)
+ * and retires the old one without freeing it, so a CUDA graph captured
+ * earlier on that stream keeps valid pointers; gqa_attn_release_workspace
+ * frees everything.  Partials of the split-KV decode kernel and of the
+ * tcgen05 kernel's key splits use the workspace; when every (batch, kv head)
+ * has one 128-row tile split into 2 to 8 CTAs and all of the grid's CTAs fit
+ * on the device at once, the tcgen05 kernel is launched as one thread-block
+ * cluster per (batch, kv head), merges its partials in distributed shared
+ * memory and allocates no workspace (gqa_attn_describe_merge tells which).
+ *
+ * CUDA graphs: a call of a given size on a stream enqueues only kernels (and
+ * allocates nothing) once a call of that size has run on that stream, so
+ * capture after one direct call.
  *
  * Returns GQA_ATTN_OK or a negative GQA_ATTN_ERR_* code.  Errors raised while
  * the kernel runs surface at the next synchronisation (CUDA convention) and,
@@ -139,8 +146,9 @@ int gqa_attn_describe(int batch, int q_len, int kv_len, int num_q_heads, int num
  * key 3: force the number of key splits of the tcgen05 kernel for units with
  *        one row tile (rounded up to even; 0 = automatic);
  * key 4: how those splits merge (0 = automatic: through distributed shared
- *        memory in one thread-block cluster per unit when the whole grid fits
- *        on the device at once; -1 = always through the workspace).
+ *        memory in one thread-block cluster per unit when a unit has 2 to 8
+ *        CTAs and the whole grid fits on the device at once; -1 = always
+ *        through the workspace).
  * A forced path that cannot run these sizes falls back to automatic.
  * Returns GQA_ATTN_OK or GQA_ATTN_ERR_ARG for an unknown key.
  */
@@ -150,13 +158,37 @@ int gqa_attn_set_override(int key, int value);
 const char* gqa_attn_error_string(int status);
 
 /*
+ * gqa_attn_describe_merge -- how gqa_attn_fwd would merge key-split partials
+ * for these sizes on the current device: *cluster = CTAs per thread-block
+ * cluster of the distributed-shared-memory merge, or 0 (workspace merge, or
+ * no splits).  Launches nothing.  Returns as gqa_attn_describe.
+ */
+int gqa_attn_describe_merge(int batch, int q_len, int kv_len, int num_q_heads, int num_kv_heads,
+                            int head_dim, int causal, int window, float softcap, int* cluster);
+
+/*
  * gqa_attn_status -- the sticky device status word of the current device
  * (GQA_ATTN_STATUS_* bits, 0 = nothing happened), read with a synchronous
  * copy; call after synchronising.  Returns -1 when it cannot be read.
- * gqa_attn_clear_status resets it to 0 and returns GQA_ATTN_OK or an error.
+ *
+ * gqa_attn_clear_status resets it to 0 and zeroes the split-ticket counters
+ * of every workspace of the current device: a kernel that gave up a bounded
+ * wait may have left a count behind, which would make a later split merge
+ * run early or never.  Call it after synchronising, with no call of this
+ * library in flight on the device, before using the device again after a
+ * non-zero status; it synchronises the device.  Returns GQA_ATTN_OK or an
+ * error.
  */
 int gqa_attn_status(void);
 int gqa_attn_clear_status(void);
+
+/*
+ * gqa_attn_release_workspace -- synchronise every device that holds a
+ * workspace of this library and free all of them (active and retired).
+ * Graphs captured before must not be replayed afterwards; the next call
+ * allocates afresh.  Returns GQA_ATTN_OK or GQA_ATTN_ERR_LAUNCH.
+ */
+int gqa_attn_release_workspace(void);
 
 /*
  * gqa_attn_selftest_bounded_wait -- failure-detection self test: launches

@@ -7,10 +7,12 @@ arguments.  Importing it does not load the library; the first call does, and
 raises if the library is missing (there is no CPU fallback).
 """
 from .attention import (attention, attention_host, clear_status, describe,  # noqa: F401
-                        make_attention, selftest_bounded_wait, set_override, status)
+                        make_attention, release_workspace, selftest_bounded_wait, set_override,
+                        status)
 from .inputs import WORKLOADS, Workload, make_inputs  # noqa: F401
 from .kv_cache import attention_ring, decode_append, kv_append  # noqa: F401
 
 __all__ = ["attention", "attention_host", "make_attention", "describe", "set_override",
-           "status", "clear_status", "selftest_bounded_wait", "WORKLOADS", "Workload",
+           "status", "clear_status", "release_workspace", "selftest_bounded_wait", "WORKLOADS",
+           "Workload",
            "make_inputs", "kv_append", "decode_append", "attention_ring"]

@@ -20,6 +20,7 @@ EXPORTS = (
     "gqa_attn_clear_status", "gqa_attn_selftest_bounded_wait",
     "gqa_attn_version", "gqa_attn_last_error_detail", "gqa_attn_fwd_static_scratch",
     "gqa_attn_kv_append", "gqa_attn_decode_append", "gqa_attn_fwd_ring",
+    "gqa_attn_describe_merge", "gqa_attn_release_workspace",
 )
 
 _I = ctypes.c_int
@@ -60,6 +61,10 @@ def load(path: str | None = None) -> ctypes.CDLL:
         lib.gqa_attn_fwd_host.argtypes = [_P] * 8 + _DIMS + [_P]
         lib.gqa_attn_describe.restype = _I
         lib.gqa_attn_describe.argtypes = _DIMS + [ctypes.POINTER(_I)] * 4
+        lib.gqa_attn_describe_merge.restype = _I
+        lib.gqa_attn_describe_merge.argtypes = _DIMS + [ctypes.POINTER(_I)]
+        lib.gqa_attn_release_workspace.restype = _I
+        lib.gqa_attn_release_workspace.argtypes = []
         lib.gqa_attn_set_override.restype = _I
         lib.gqa_attn_set_override.argtypes = [_I, _I]
         lib.gqa_attn_error_string.restype = ctypes.c_char_p

@@ -129,7 +129,12 @@ def describe(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, causal=F
                                        head_dim, c, w, s, *[ctypes.byref(o) for o in outs])
     _lib.check(rc, "gqa_attn_describe")
     path = {0: "none", 1: "decode", 2: "prefill", 3: "zero"}[outs[0].value]
-    return dict(path=path, splits=outs[1].value, ctas=outs[2].value, tiles=outs[3].value)
+    cluster = ctypes.c_int(0)
+    rc = _lib.load().gqa_attn_describe_merge(batch, q_len, kv_len, num_q_heads, num_kv_heads,
+                                             head_dim, c, w, s, ctypes.byref(cluster))
+    _lib.check(rc, "gqa_attn_describe_merge")
+    return dict(path=path, splits=outs[1].value, ctas=outs[2].value, tiles=outs[3].value,
+                cluster=cluster.value)
 
 
 def set_override(key: str, value: int) -> None:
@@ -148,7 +153,13 @@ def status() -> int:
 
 
 def clear_status() -> None:
+    """Reset the status word and the split-ticket counters (after a sync)."""
     _lib.check(_lib.load().gqa_attn_clear_status(), "gqa_attn_clear_status")
+
+
+def release_workspace() -> None:
+    """Free every split workspace the library holds (synchronises)."""
+    _lib.check(_lib.load().gqa_attn_release_workspace(), "gqa_attn_release_workspace")
 
 
 def selftest_bounded_wait(limit_us: int = 1000, stream=None) -> None:

@@ -14,6 +14,7 @@
 #include <map>
 #include <mutex>
 #include <utility>
+#include <vector>
 
 #include "gqa_attn.h"
 #include "status.cuh"
@@ -300,47 +301,52 @@ struct Workspace {
   size_t ticket_bytes = 0;
 };
 std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+// Buffers replaced by bigger ones: kept, not freed, because a CUDA graph
+// captured earlier may still reference them (freed by
+// gqa_attn_release_workspace).  Tickets are listed with their size so that
+// gqa_attn_clear_status can zero them too.
+struct Retired {
+  int dev;
+  void* ptr;
+  size_t ticket_bytes;  // > 0: a ticket buffer
+};
+std::vector<Retired> g_retired;
 
 // Workspace for (current device, stream): `bytes` of scratch for the split
 // partials and `ticket_bytes` of ticket counters.  Tickets live in their own
 // buffer, cleared on allocation; every kernel leaves its tickets at zero.
+// Growing allocates new buffers (no synchronisation) and retires the old.
 int get_workspace(cudaStream_t stream, size_t bytes, size_t ticket_bytes, void** out,
                   void** tickets) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ATTN_ERR_DEVICE;
   std::lock_guard<std::mutex> lk(g_mu);
   Workspace& ws = g_ws[std::make_pair(dev, stream)];
-  if (ws.bytes < bytes || ws.ticket_bytes < ticket_bytes) {
-    if (ws.ptr || ws.tickets) {
-      cudaStreamSynchronize(stream);
-      if (ws.bytes < bytes && ws.ptr) {
-        cudaFree(ws.ptr);
-        ws.ptr = nullptr;
-        ws.bytes = 0;
-      }
-      if (ws.ticket_bytes < ticket_bytes && ws.tickets) {
-        cudaFree(ws.tickets);
-        ws.tickets = nullptr;
-        ws.ticket_bytes = 0;
-      }
+  if (ws.bytes < bytes) {
+    void* p = nullptr;
+    const size_t want = bytes + bytes / 4;
+    if (cudaMalloc(&p, want) != cudaSuccess) {
+      cudaGetLastError();
+      return GQA_ATTN_ERR_ALLOC;
     }
-    if (!ws.ptr) {
-      const size_t want = bytes + bytes / 4;
-      if (cudaMalloc(&ws.ptr, want) != cudaSuccess) {
-        cudaGetLastError();
-        return GQA_ATTN_ERR_ALLOC;
-      }
-      ws.bytes = want;
+    if (ws.ptr) g_retired.push_back({dev, ws.ptr, 0});
+    ws.ptr = p;
+    ws.bytes = want;
+  }
+  if (ws.ticket_bytes < ticket_bytes) {
+    void* p = nullptr;
+    const size_t want = ticket_bytes < 4096 ? 4096 : ticket_bytes * 2;
+    if (cudaMalloc(&p, want) != cudaSuccess) {
+      cudaGetLastError();
+      return GQA_ATTN_ERR_ALLOC;
     }
-    if (!ws.tickets) {
-      const size_t want = ticket_bytes < 4096 ? 4096 : ticket_bytes * 2;
-      if (cudaMalloc(&ws.tickets, want) != cudaSuccess) {
-        cudaGetLastError();
-        return GQA_ATTN_ERR_ALLOC;
-      }
-      if (cudaMemsetAsync(ws.tickets, 0, want, stream) != cudaSuccess) return GQA_ATTN_ERR_LAUNCH;
-      ws.ticket_bytes = want;
+    if (cudaMemsetAsync(p, 0, want, stream) != cudaSuccess) {
+      cudaFree(p);
+      return GQA_ATTN_ERR_LAUNCH;
     }
+    if (ws.tickets) g_retired.push_back({dev, ws.tickets, ws.ticket_bytes});
+    ws.tickets = p;
+    ws.ticket_bytes = want;
   }
   *out = ws.ptr;
   *tickets = ws.tickets;
@@ -405,6 +411,7 @@ int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
                      cudaStream_t stream) {
   using C = DecodeCfg<KS>;
   const int slot = (KS / 4 - 1) + (kT ? 4 : 0);
+  std::unique_lock<std::mutex> lk(g_mu);
   if (!dev.decode_attr[slot]) {
     cudaError_t e = cudaFuncSetAttribute(decode_splitkv_kernel<KS, kT>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -416,6 +423,7 @@ int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(decode)", e, GQA_ATTN_ERR_LAUNCH);
     dev.decode_attr[slot] = true;
   }
+  lk.unlock();
   CUtensorMap tk, tv;
   if (encode_kv_map(&tk, k, pr, kDecTile) != GQA_ATTN_OK ||
       encode_kv_map(&tv, v, pr, kDecTile) != GQA_ATTN_OK)
@@ -481,29 +489,102 @@ int launch_decode(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void
   }
 }
 
+// Softcap degree of the tcgen05 kernel's tanh polynomial: caps up to
+// kTanh5MaxCap take degree 5, larger caps degree 7, 0 = no softcap.
+int cap_degree(const Problem& pr) {
+  return pr.softcap > 0.f ? (pr.softcap <= kTanh5MaxCap ? 5 : 7) : 0;
+}
+
 template <int DCH, int kCapDeg, bool kSplit>
-int launch_prefill_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
-                     const void* k, const void* v, void* o, void* ws, void* tickets,
-                     cudaStream_t stream) {
+constexpr int prefill_slot() {
+  return (DCH - 1) + (kCapDeg == 5 ? 2 : kCapDeg == 7 ? 4 : 0) + (kSplit ? 6 : 0);
+}
+
+// One-time per device and instantiation (under g_mu): the register-split
+// check and the dynamic shared memory limit.
+template <int DCH, int kCapDeg, bool kSplit>
+int prefill_setup(DeviceInfo& dev) {
+  using C = PrefillCfg<DCH>;
+  constexpr int attr = prefill_slot<DCH, kCapDeg, kSplit>();
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (dev.prefill_attr[attr]) return GQA_ATTN_OK;
+  // The register split inside the kernel must fit what the block is
+  // launched with, or setmaxnreg.inc could never be granted.
+  cudaFuncAttributes fa;
+  const cudaError_t ea = cudaFuncGetAttributes(&fa, prefill_sm100_kernel<DCH, kCapDeg, kSplit>);
+  if (ea != cudaSuccess) return cuda_fail("cudaFuncGetAttributes(prefill)", ea, GQA_ATTN_ERR_LAUNCH);
+  if ((long long)fa.numRegs * kPfThreads < kRegSplitTotal) {
+    snprintf(g_detail, sizeof g_detail, "prefill kernel built with %d registers/thread: "
+             "register split needs %d", fa.numRegs, kRegSplitTotal);
+    return GQA_ATTN_ERR_LAUNCH;
+  }
+  const cudaError_t e = cudaFuncSetAttribute(prefill_sm100_kernel<DCH, kCapDeg, kSplit>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
+  if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(prefill)", e, GQA_ATTN_ERR_LAUNCH);
+  dev.prefill_attr[attr] = true;
+  return GQA_ATTN_OK;
+}
+
+// Paired key splits, one item per CTA: a cluster per unit merges its
+// partials through distributed shared memory when every cluster of the grid
+// can be resident at once (one wave) and a unit has 2..8 CTAs; *csize gets
+// the CTAs per cluster, or 0 for the workspace merge.
+template <int DCH, int kCapDeg>
+int prefill_cluster_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, int* csize) {
+  using C = PrefillCfg<DCH>;
+  *csize = 0;
+  if (!pl.split_pairs || g_no_cluster.load()) return GQA_ATTN_OK;
+  const int half = pl.splits / 2;
+  if (half < 2 || half > 8 || pl.ctas != pr.units * half) return GQA_ATTN_OK;
+  int rc = prefill_setup<DCH, kCapDeg, true>(dev);
+  if (rc != GQA_ATTN_OK) return rc;
+  constexpr int attr = prefill_slot<DCH, kCapDeg, true>();
+  std::lock_guard<std::mutex> lk(g_mu);
+  int& fit = dev.cluster_max[attr][half];
+  if (fit < 0) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)half;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)pl.ctas);
+    cfg.blockDim = dim3(kPfThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, prefill_sm100_kernel<DCH, kCapDeg, true>, &cfg) !=
+        cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    fit = n;
+  }
+  if (fit >= pr.units) *csize = half;
+  return GQA_ATTN_OK;
+}
+
+int prefill_cluster(const Problem& pr, const Plan& pl, DeviceInfo& dev, int* csize) {
+  const int deg = cap_degree(pr);
+  if (pl.dch == 1)
+    return deg == 5 ? prefill_cluster_k<1, 5>(pr, pl, dev, csize)
+         : deg == 7 ? prefill_cluster_k<1, 7>(pr, pl, dev, csize)
+                    : prefill_cluster_k<1, 0>(pr, pl, dev, csize);
+  return deg == 5 ? prefill_cluster_k<2, 5>(pr, pl, dev, csize)
+       : deg == 7 ? prefill_cluster_k<2, 7>(pr, pl, dev, csize)
+                  : prefill_cluster_k<2, 0>(pr, pl, dev, csize);
+}
+
+template <int DCH, int kCapDeg, bool kSplit>
+int launch_prefill_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, int csize,
+                     const void* q, const void* k, const void* v, void* o, void* ws,
+                     void* tickets, cudaStream_t stream) {
   using C = PrefillCfg<DCH>;
   constexpr bool kCap = kCapDeg != 0;
-  constexpr int attr = (DCH - 1) + (kCapDeg == 5 ? 2 : kCapDeg == 7 ? 4 : 0) + (kSplit ? 6 : 0);
-  if (!dev.prefill_attr[attr]) {
-    // The register split inside the kernel must fit what the block is
-    // launched with, or setmaxnreg.inc could never be granted.
-    cudaFuncAttributes fa;
-    const cudaError_t ea = cudaFuncGetAttributes(&fa, prefill_sm100_kernel<DCH, kCapDeg, kSplit>);
-    if (ea != cudaSuccess) return cuda_fail("cudaFuncGetAttributes(prefill)", ea, GQA_ATTN_ERR_LAUNCH);
-    if ((long long)fa.numRegs * kPfThreads < kRegSplitTotal) {
-      snprintf(g_detail, sizeof g_detail, "prefill kernel built with %d registers/thread: "
-               "register split needs %d", fa.numRegs, kRegSplitTotal);
-      return GQA_ATTN_ERR_LAUNCH;
-    }
-    const cudaError_t e = cudaFuncSetAttribute(
-        prefill_sm100_kernel<DCH, kCapDeg, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(prefill)", e, GQA_ATTN_ERR_LAUNCH);
-    dev.prefill_attr[attr] = true;
-  }
+  int rc = prefill_setup<DCH, kCapDeg, kSplit>(dev);
+  if (rc != GQA_ATTN_OK) return rc;
   CUtensorMap tq, tk, tv, to;
   if (encode_map(&tq, q, pr.d, pr.rows, pr.units, kPfM) != GQA_ATTN_OK ||
       encode_map(&to, o, pr.d, pr.rows, pr.units, 32) != GQA_ATTN_OK ||
@@ -528,45 +609,14 @@ int launch_prefill_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.tickets = (unsigned int*)tickets;
   p.pair_heads = pl.pair_heads;
   p.heavy_first = (pr.causal || pr.window > 0) && !pl.split_pairs ? 1 : 0;
-  // Paired key splits, one item per CTA: a cluster per unit merges its
-  // partials through distributed shared memory, when every cluster of the
-  // grid can be resident at once (one wave); otherwise the workspace merge.
-  int csize = 0;
-  if (kSplit && pl.split_pairs && !g_no_cluster.load()) {
-    const int half = pl.splits / 2;
-    if (half >= 2 && half <= 8 && pl.ctas == pr.units * half) {
-      int& fit = dev.cluster_max[attr][half];
-      if (fit < 0) {
-        cudaLaunchConfig_t cfg = {};
-        cudaLaunchAttribute at[1];
-        at[0].id = cudaLaunchAttributeClusterDimension;
-        at[0].val.clusterDim.x = (unsigned)half;
-        at[0].val.clusterDim.y = 1;
-        at[0].val.clusterDim.z = 1;
-        cfg.gridDim = dim3((unsigned)pl.ctas);
-        cfg.blockDim = dim3(kPfThreads);
-        cfg.dynamicSmemBytes = C::kSmemBytes;
-        cfg.attrs = at;
-        cfg.numAttrs = 1;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, prefill_sm100_kernel<DCH, kCapDeg, kSplit>, &cfg) !=
-            cudaSuccess) {
-          (void)cudaGetLastError();
-          n = 0;
-        }
-        fit = n;
-      }
-      if (fit >= pr.units) csize = half;
-    }
-  }
-  p.cluster_merge = csize;
+  p.cluster_merge = kSplit ? csize : 0;
   p.causal = pr.causal;
   p.window = pr.window;
   const float rs = 1.0f / std::sqrt((float)pr.d);
   p.logit_scale = kLog2e * rs;
   p.cap_in = kCap ? rs / pr.softcap : 0.f;
   p.cap_out = kCap ? pr.softcap * kLog2e : 0.f;
-  if (csize > 0) {
+  if (p.cluster_merge > 0) {
     // One item per CTA, clusters of csize consecutive CTAs (one unit each).
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
@@ -593,26 +643,25 @@ int launch_prefill_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
 }
 
 template <int DCH, int kCapDeg>
-int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
-                     const void* k, const void* v, void* o, void* ws, void* tickets,
-                     cudaStream_t stream) {
+int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, int csize,
+                     const void* q, const void* k, const void* v, void* o, void* ws,
+                     void* tickets, cudaStream_t stream) {
   return pl.splits > 1
-             ? launch_prefill_k<DCH, kCapDeg, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
-             : launch_prefill_k<DCH, kCapDeg, false>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+             ? launch_prefill_k<DCH, kCapDeg, true>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
+             : launch_prefill_k<DCH, kCapDeg, false>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream);
 }
 
-int launch_prefill(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
+int launch_prefill(const Problem& pr, const Plan& pl, DeviceInfo& dev, int csize, const void* q,
                    const void* k, const void* v, void* o, void* ws, void* tickets,
                    cudaStream_t stream) {
-  // Softcaps up to kTanh5MaxCap take the degree-5 tanh polynomial.
-  if (pr.softcap > 0.f && pr.softcap <= kTanh5MaxCap)
-    return pl.dch == 1 ? launch_prefill_d<1, 5>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
-                       : launch_prefill_d<2, 5>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
-  if (pr.softcap > 0.f)
-    return pl.dch == 1 ? launch_prefill_d<1, 7>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
-                       : launch_prefill_d<2, 7>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
-  return pl.dch == 1 ? launch_prefill_d<1, 0>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
-                     : launch_prefill_d<2, 0>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+  const int deg = cap_degree(pr);
+  if (pl.dch == 1)
+    return deg == 5 ? launch_prefill_d<1, 5>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
+         : deg == 7 ? launch_prefill_d<1, 7>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
+                    : launch_prefill_d<1, 0>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream);
+  return deg == 5 ? launch_prefill_d<2, 5>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
+       : deg == 7 ? launch_prefill_d<2, 7>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
+                  : launch_prefill_d<2, 0>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream);
 }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
@@ -673,13 +722,20 @@ int run(const Problem& pr, const void* q, const void* k, const void* v, void* o,
                                                                  : GQA_ATTN_ERR_LAUNCH;
     }
     default: {
+      // Key splits merged in distributed shared memory need no workspace.
+      int csize = 0;
+      if (pl.path == kPathPrefill && pl.splits > 1) {
+        rc = prefill_cluster(pr, pl, *dev, &csize);
+        if (rc != GQA_ATTN_OK) return rc;
+      }
       void* ws = nullptr;
       void* tickets = nullptr;
-      if (pl.ws_bytes) {
+      if (pl.ws_bytes && csize == 0) {
         rc = get_workspace(stream, pl.ws_bytes, pl.ticket_bytes, &ws, &tickets);
         if (rc != GQA_ATTN_OK) return rc;
       }
-      if (pl.path == kPathPrefill) return launch_prefill(pr, pl, *dev, q, k, v, o, ws, tickets, stream);
+      if (pl.path == kPathPrefill)
+        return launch_prefill(pr, pl, *dev, csize, q, k, v, o, ws, tickets, stream);
       return launch_decode(pr, pl, *dev, q, k, v, o, ws, tickets, stream);
     }
   }
@@ -827,8 +883,66 @@ int gqa_attn_status(void) {
 
 int gqa_attn_clear_status(void) {
   const uint32_t z = 0;
-  return cudaMemcpyToSymbol(gqa::g_gqa_status, &z, sizeof z) == cudaSuccess ? GQA_ATTN_OK
-                                                                             : GQA_ATTN_ERR_LAUNCH;
+  if (cudaMemcpyToSymbol(gqa::g_gqa_status, &z, sizeof z) != cudaSuccess) return GQA_ATTN_ERR_LAUNCH;
+  // A kernel that gave up a wait may have left split tickets counted, which
+  // would make the next merge on that buffer start early or never: zero
+  // every ticket buffer of this device (active and retired).
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GQA_ATTN_ERR_DEVICE;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (auto& kv : g_ws)
+      if (kv.first.first == dev && kv.second.tickets &&
+          cudaMemset(kv.second.tickets, 0, kv.second.ticket_bytes) != cudaSuccess)
+        return GQA_ATTN_ERR_LAUNCH;
+    for (const Retired& r : g_retired)
+      if (r.dev == dev && r.ticket_bytes > 0 && cudaMemset(r.ptr, 0, r.ticket_bytes) != cudaSuccess)
+        return GQA_ATTN_ERR_LAUNCH;
+  }
+  return cudaDeviceSynchronize() == cudaSuccess ? GQA_ATTN_OK : GQA_ATTN_ERR_LAUNCH;
+}
+
+int gqa_attn_release_workspace(void) {
+  int cur = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return GQA_ATTN_ERR_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  int rc = GQA_ATTN_OK;
+  auto release = [&](int dev, void* p) {
+    if (!p) return;
+    if (cudaSetDevice(dev) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess ||
+        cudaFree(p) != cudaSuccess)
+      rc = GQA_ATTN_ERR_LAUNCH;
+  };
+  for (auto& kv : g_ws) {
+    release(kv.first.first, kv.second.ptr);
+    release(kv.first.first, kv.second.tickets);
+  }
+  g_ws.clear();
+  for (const Retired& r : g_retired) release(r.dev, r.ptr);
+  g_retired.clear();
+  if (cudaSetDevice(cur) != cudaSuccess) rc = GQA_ATTN_ERR_DEVICE;
+  return rc;
+}
+
+int gqa_attn_describe_merge(int batch, int q_len, int kv_len, int num_q_heads, int num_kv_heads,
+                            int head_dim, int causal, int window, float softcap, int* cluster) {
+  Problem pr;
+  int rc = validate(batch, q_len, kv_len, num_q_heads, num_kv_heads, head_dim, causal, window,
+                    softcap, &pr);
+  if (rc != GQA_ATTN_OK) return rc;
+  DeviceInfo* dev = nullptr;
+  rc = device_info(&dev);
+  if (rc != GQA_ATTN_OK) return rc;
+  Plan pl;
+  rc = make_plan(pr, *dev, &pl);
+  if (rc != GQA_ATTN_OK) return rc;
+  int csize = 0;
+  if (pl.path == kPathPrefill && pl.splits > 1) {
+    rc = prefill_cluster(pr, pl, *dev, &csize);
+    if (rc != GQA_ATTN_OK) return rc;
+  }
+  if (cluster) *cluster = csize;
+  return GQA_ATTN_OK;
 }
 
 int gqa_attn_selftest_bounded_wait(int limit_us, void* stream) {
@@ -841,7 +955,7 @@ int gqa_attn_selftest_bounded_wait(int limit_us, void* stream) {
   return cudaGetLastError() == cudaSuccess ? GQA_ATTN_OK : GQA_ATTN_ERR_LAUNCH;
 }
 
-int gqa_attn_version(void) { return 200; }
+int gqa_attn_version(void) { return 300; }
 
 // Argument checks of a KV-cache append (nothing launched).  *n_out gets the
 // number of new elements per tensor; GQA_ATTN_OK with *n_out == 0 means

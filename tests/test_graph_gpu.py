@@ -40,3 +40,43 @@ def test_captured_call_replays_like_a_direct_call(w):
         torch.cuda.synchronize()
         assert torch.equal(out, want)
     assert mgq.status() & 0x1f == 0
+
+
+def test_captured_call_survives_workspace_growth():
+    # A graph captured with a small split call keeps valid workspace
+    # pointers after a larger direct call on the same stream grows the
+    # stream's workspace (the old buffers are retired, not freed).
+    from oracle import oracle
+
+    small = Workload("small", 1, 1, 4000, 8, 2, 128, True, None, None, 41)
+    big = Workload("big", 16, 1, 60000, 32, 8, 128, True, None, None, 42)
+    q, k, v = (t.cuda() for t in make_inputs(small))
+    out = torch.empty_like(q)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        mgq.attention(q, k, v, causal=True, out=out)
+    s.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        mgq.attention(q, k, v, causal=True, out=out)
+    qb, kb, vb = (t.cuda() for t in make_inputs(big))
+    plan_s = mgq.describe(1, 1, 4000, 8, 2, 128, True)
+    plan_b = mgq.describe(16, 1, 60000, 32, 8, 128, True)
+    assert plan_s["splits"] > 1 and plan_b["splits"] * plan_b["ctas"] > plan_s["splits"] * plan_s["ctas"]
+    with torch.cuda.stream(s):
+        ob = mgq.attention(qb, kb, vb, causal=True)   # grows the stream's workspace
+    s.synchronize()
+    q2, k2, v2 = make_inputs(small, seed=143)
+    q.copy_(q2)
+    k.copy_(k2)
+    v.copy_(v2)
+    with torch.cuda.stream(s):
+        g.replay()
+    s.synchronize()
+    want = oracle.attention(q2, k2, v2, causal=True, window=None, softcap=None)
+    got = out.float().cpu().numpy()
+    assert abs(got - want).max() <= 2e-2 and ((abs(got - want) <= 2e-2 + 2e-2 * abs(want)).all())
+    assert torch.isfinite(ob).all()
+    del g
+    assert mgq.status() & 0x1f == 0
