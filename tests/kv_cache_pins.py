@@ -8,6 +8,8 @@ it) and raises AssertionError on a mismatch.  They pin it to:
 * a library routine: torch's float32 -> bfloat16 conversion on values of
   every magnitude, including exact ties;
 * the hand-worked updates of ``golden/kv_update_hand_examples.json``;
+* the three worked examples the page prints ("KV Cache Update at a
+  Position", "Examples"), in ``golden/kv_update_page_examples.json``;
 * invariants of the update ("KV Cache Update at a Position", TensorTonic):
   slots outside [position, position + L) are untouched bit for bit, the new
   block equals the converted new vectors concatenated after the old prefix,
@@ -28,6 +30,8 @@ import torch
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
                       "kv_update_hand_examples.json")
+PAGE_EXAMPLES = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                             "kv_update_page_examples.json")
 
 
 def _f32(x):
@@ -84,8 +88,8 @@ def _widen(a, kc):
     return kc.bf16_bits_to_f32(a) if a.dtype == np.uint16 else a
 
 
-def pin_hand_examples(kc):
-    with open(GOLDEN) as f:
+def pin_hand_examples(kc, path=GOLDEN):
+    with open(path) as f:
         cases = json.load(f)["cases"]
     for c in cases:
         k0 = _as_cache(c["key_cache"], c["cache_dtype"], kc)
@@ -98,6 +102,11 @@ def pin_hand_examples(kc):
             assert np.array_equal(g, w), f"{c['name']}: {g.tolist()} != {w.tolist()}"
             assert np.array_equal(np.signbit(g), np.signbit(w)), f"{c['name']}: zero signs"
         assert k1.dtype == k0.dtype and k1.shape == k0.shape
+
+
+def pin_page_examples(kc):
+    """The page's printed inputs give the page's printed outputs."""
+    pin_hand_examples(kc, PAGE_EXAMPLES)
 
 
 def pin_update_invariants(kc):
@@ -159,5 +168,5 @@ def pin_ring_replays_sequence(kc):
 
 
 ALL_PINS = [pin_rounding_closed_forms, pin_rounding_matches_torch, pin_round_trip_identity,
-            pin_hand_examples, pin_update_invariants, pin_ring_hand_example,
+            pin_hand_examples, pin_page_examples, pin_update_invariants, pin_ring_hand_example,
             pin_ring_replays_sequence]

@@ -93,6 +93,34 @@ def test_append_bit_exact(combo, shape):
     assert_same_bits(bits_of(from_layout(vc.cpu(), not seq_major)), want_v, "value cache")
 
 
+def test_append_page_examples():
+    # The three worked examples printed on "KV Cache Update at a Position"
+    # ("Examples": fp32 caches (B, S, H, D), fp32 new vectors), through the
+    # append kernel.  Its head_dim is a multiple of 8, so each example's
+    # vectors are zero-padded to 8 columns: the padded result must be the
+    # page's output, padded the same way.
+    import json
+
+    from .kv_cache_pins import PAGE_EXAMPLES
+
+    def pad8(a):
+        a = np.asarray(a, dtype=np.float32)
+        out = np.zeros(a.shape[:-1] + (8,), np.float32)
+        out[..., :a.shape[-1]] = a
+        return torch.from_numpy(out)
+
+    with open(PAGE_EXAMPLES) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        kc, vc = pad8(c["key_cache"]).cuda(), pad8(c["value_cache"]).cuda()
+        n = mgq.kv_append(kc, vc, pad8(c["new_keys"]).cuda(), pad8(c["new_values"]).cuda(),
+                          c["position"])
+        torch.cuda.synchronize()
+        assert n == c["expected_length"], c["name"]
+        assert torch.equal(kc.cpu(), pad8(c["expected_key_cache"])), c["name"]
+        assert torch.equal(vc.cpu(), pad8(c["expected_value_cache"])), c["name"]
+
+
 def test_append_edges():
     x = make_cache_inputs(2, 16, 2, 64, 16, seed=9)
     kc, vc = x["k_cache"].cuda(), x["v_cache"].cuda()

@@ -6,8 +6,8 @@ cause -- so this variant of the split-KV decode path keeps its split
 partials and tickets in one fixed device array inside the library instead of
 a workspace allocated on first need.  These tests call it through the C ABI,
 twice in a row (the array keeps the previous call's contents), and compare
-each result with gqa_attn_fwd's within the parity tolerance
-(rtol = atol = 2e-2).  This file is collected last on purpose.
+each result with gqa_attn_fwd's and with the fp64 oracle, within the parity
+tolerance (rtol = atol = 2e-2).  This file is collected last on purpose.
 """
 import ctypes
 
@@ -17,6 +17,7 @@ import torch
 
 from masked_grouped_query_b200 import _lib
 from masked_grouped_query_b200.inputs import Workload, make_inputs
+from oracle import oracle
 
 pytestmark = pytest.mark.gpu
 
@@ -43,7 +44,9 @@ CASES = [
 @pytest.mark.parametrize("w", CASES, ids=[c.name for c in CASES])
 def test_static_scratch_matches_gqa_attn_fwd_twice(w):
     lib = _lib.load()
-    q, k, v = (t.cuda() for t in make_inputs(w))
+    qh, kh, vh = make_inputs(w)
+    exact = oracle.attention(qh, kh, vh, causal=w.causal, window=w.window, softcap=w.softcap)
+    q, k, v = qh.cuda(), kh.cuda(), vh.cuda()
     ref = torch.empty_like(q)
     assert _call(lib.gqa_attn_fwd, w, q, k, v, ref) == 0
     torch.cuda.synchronize()
@@ -56,6 +59,8 @@ def test_static_scratch_matches_gqa_attn_fwd_twice(w):
         got = out.float().cpu().numpy()
         assert np.isfinite(got).all()
         np.testing.assert_allclose(got, want, rtol=2e-2, atol=2e-2)
+        # and against the oracle: elementwise |got - exact| <= 2e-2 + 2e-2 |exact|
+        np.testing.assert_allclose(got, exact, rtol=2e-2, atol=2e-2)
     assert lib.gqa_attn_status() & 0x1f == 0
 
 
