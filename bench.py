@@ -141,6 +141,41 @@ def ncu_traffic(workload: str):
     return e.get("dram_bytes_per_launch")
 
 
+def roofline_block(w: Workload, ms_mean: float, pk: dict, pk_src: str) -> dict:
+    """Roofline of one attention workload timed at ``ms_mean`` ms per call:
+    HBM for decode-class workloads (algorithmic K/V bytes), bf16 tensor peak
+    otherwise (FLOPs over unmasked pairs)."""
+    _, unit, work = metric_of(w)
+    if unit == "GB/s":
+        bound, peak = "hbm", pk["hbm_gbs"]
+    else:
+        bound, peak = "tensor", pk["bf16_tflops"]
+    achieved = work / (ms_mean * 1e-3)
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak,
+            "peak_source": f"{pk_src} (MEASURED_PEAKS.json)" if pk_src == "measured" else "fallback",
+            "traffic": ncu_traffic(w.name)}
+
+
+def workload_entry(w: Workload, res: dict, pk: dict, pk_src: str) -> dict:
+    """One attention workload's figures from a timing result of _timed_loop."""
+    name, unit, work = metric_of(w)
+    return {"metric": name, "value": work / (res["ms_mean"] * 1e-3), "unit": unit,
+            "ms_mean": res["ms_mean"], "ms_median": res["ms_median"],
+            "ms_p10": res["ms_p10"], "ms_p90": res["ms_p90"],
+            "config": {k: v for k, v in w.cfg().items() if k != "name"},
+            "roofline": roofline_block(w, res["ms_mean"], pk, pk_src),
+            "gpu_launches": res.get("launches"), "plan": res.get("plan"),
+            "device_status": res.get("status")}
+
+
+def other_workloads(main_name: str, timer, pk: dict, pk_src: str) -> dict:
+    """Every attention workload except ``main_name``, each timed by
+    ``timer(w)`` (the same L2 flush and CUDA-event timing as the headline)."""
+    return {w.name: workload_entry(w, timer(w), pk, pk_src)
+            for w in WORKLOADS.values() if w.name != main_name}
+
+
 # ------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -481,7 +516,10 @@ def main():
                     help="an attention workload, or one of the KV-cache / ring extras "
                          "(timed alone: one JSON line with its roofline, 1 GPU)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--all", action="store_true", help="also time every other workload")
+    ap.add_argument("--all", action="store_true",
+                    help="also time the KV-cache, ring-window and append extras")
+    ap.add_argument("--no-others", action="store_true",
+                    help="skip the other attention workloads (timed by default at N = 1)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     args = ap.parse_args()
@@ -544,16 +582,15 @@ def main():
     value = work * ctx.world / (ms * 1e-3)
 
     extra = {}
+    others_clocks = None
+    if ctx.world == 1 and not args.no_others:
+        # The other configurations of the metric, each timed like the headline.
+        with ClockSampler(gpu_index) as clk2:
+            extra = other_workloads(
+                w.name, lambda o: time_native(o, args.steps, args.warmup, device, _NoDist()),
+                pk, pk_src)
+        others_clocks = clk2.summary()
     if args.all and ctx.rank == 0:
-        for other in WORKLOADS.values():
-            if other.name == w.name:
-                continue
-            r = time_native(other, max(20, args.steps // 4), args.warmup, device, _NoDist())
-            n2, u2, wk2 = metric_of(other)
-            a = wk2 / (r["ms_mean"] * 1e-3)
-            pkv = pk["hbm_gbs"] if u2 == "GB/s" else pk["bf16_tflops"]
-            extra[other.name] = {"metric": n2, "value": a, "unit": u2, "ms": r["ms_mean"],
-                                 "frac_of_peak": a / pkv, "plan": r["plan"]}
         for st in CACHE_STEPS.values():
             r = time_cache_step(st, max(20, args.steps // 4), args.warmup, device, _NoDist())
             a = r["bytes"] / 1e9 / (r["ms_mean"] * 1e-3)
@@ -575,17 +612,7 @@ def main():
             "shape": "batch 2, 4096 tokens, 4 kv heads, head_dim 128, (B,S,H,D) cache"}
 
     if ctx.rank == 0:
-        if unit == "GB/s":
-            peak = pk["hbm_gbs"]
-            roof = {"bound": "hbm", "achieved": work / (res["ms_mean"] * 1e-3), "peak": peak,
-                    "unit": "GB/s"}
-        else:
-            peak = pk["bf16_tflops"]
-            roof = {"bound": "tensor", "achieved": work / (res["ms_mean"] * 1e-3), "peak": peak,
-                    "unit": "TFLOP/s"}
-        roof["frac"] = roof["achieved"] / roof["peak"]
-        roof["peak_source"] = f"{pk_src} (MEASURED_PEAKS.json)" if pk_src == "measured" else "fallback"
-        roof["traffic"] = ncu_traffic(w.name)
+        roof = roofline_block(w, res["ms_mean"], pk, pk_src)
         line = {"metric": name, "value": value, "unit": unit, "n_gpus": ctx.world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -610,6 +637,8 @@ def main():
                                     "kind": "oracle", "sample": desc, "cpu": cpu_model()}
         if extra:
             line["other_workloads"] = extra
+        if others_clocks is not None:
+            line["other_workloads_clocks"] = others_clocks
         print(json.dumps(line))
     ctx.close()
 

@@ -59,3 +59,30 @@ def test_source_hash_ignores_comments_only(tmp_path):
 def test_metric_units(name):
     metric, unit, work = bench.metric_of(WORKLOADS[name])
     assert unit in ("GB/s", "TFLOP/s") and work > 0
+
+
+def test_default_run_reports_every_other_config_with_its_roofline():
+    # The headline is one workload; the other four configurations of the
+    # metric come with the same timing fields and a roofline block each.
+    pk = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0}
+    seen = []
+
+    def timer(w):  # stands in for the CUDA-event loop
+        seen.append(w.name)
+        return {"ms_mean": 0.1, "ms_median": 0.09, "ms_p10": 0.08, "ms_p90": 0.12,
+                "launches": 20, "plan": {"path": 2}, "status": 0}
+
+    out = bench.other_workloads("gqa_decode", timer, pk, "fallback")
+    assert sorted(out) == sorted(n for n in WORKLOADS if n != "gqa_decode") == sorted(seen)
+    for name, e in out.items():
+        w = WORKLOADS[name]
+        _, unit, work = bench.metric_of(w)
+        roof = e["roofline"]
+        assert e["unit"] == roof["unit"] == unit
+        assert roof["bound"] == ("hbm" if unit == "GB/s" else "tensor")
+        assert roof["peak"] == (pk["hbm_gbs"] if unit == "GB/s" else pk["bf16_tflops"])
+        assert abs(roof["achieved"] - work / 1e-4) < 1e-6 * roof["achieved"]
+        assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-12
+        assert e["value"] == roof["achieved"]
+        assert e["ms_median"] == 0.09 and e["gpu_launches"] == 20
+        assert "traffic" in roof
