@@ -38,6 +38,7 @@ struct DeviceInfo {
   int smem_optin = 0;
   bool decode_attr[8] = {false, false, false, false, false, false, false, false};
   bool prefill_attr[12] = {};  // per (DCH, softcap degree, split) instantiation
+  int append_blocks[4] = {};    // resident kv_append blocks per SM, per instantiation
   // Clusters of n CTAs of a split instantiation that can be resident at once
   // (cudaOccupancyMaxActiveClusters); -1 = not asked yet.
   int cluster_max[12][9];
@@ -1025,14 +1026,31 @@ int gqa_attn_kv_append(void* k_cache, void* v_cache, const void* new_k, const vo
   p.new_head_major = (flags & GQA_KV_NEW_HEAD_MAJOR) ? 1 : 0;
   p.ring = ring ? 1 : 0;
   const long long chunks = 2 * n / 8;  // 8 elements per thread, keys then values
-  long long blocks = (chunks + 255) / 256;
-  if (blocks > 8LL * dev->sms) blocks = 8LL * dev->sms;
   cudaStream_t st = (cudaStream_t)stream;
   const bool nf = !(flags & GQA_KV_NEW_BF16), cf = (flags & GQA_KV_CACHE_F32) != 0;
-  if (nf && cf) kv_append_kernel<true, true><<<(unsigned)blocks, 256, 0, st>>>(p);
-  else if (nf) kv_append_kernel<true, false><<<(unsigned)blocks, 256, 0, st>>>(p);
-  else if (cf) kv_append_kernel<false, true><<<(unsigned)blocks, 256, 0, st>>>(p);
-  else kv_append_kernel<false, false><<<(unsigned)blocks, 256, 0, st>>>(p);
+  // One wave: as many blocks as are resident at once (the grid-stride loop
+  // takes the rest), so no second partial wave trails the first.
+  const int slot = (nf ? 2 : 0) + (cf ? 1 : 0);
+  void (*const kern[4])(const KvAppendParams) = {
+      kv_append_kernel<false, false>, kv_append_kernel<false, true>,
+      kv_append_kernel<true, false>, kv_append_kernel<true, true>};
+  int per_sm;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (dev->append_blocks[slot] <= 0) {
+      int nb = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern[slot], 256, 0) != cudaSuccess ||
+          nb < 1) {
+        (void)cudaGetLastError();
+        nb = 1;
+      }
+      dev->append_blocks[slot] = nb;
+    }
+    per_sm = dev->append_blocks[slot];
+  }
+  long long blocks = (chunks + 255) / 256;
+  if (blocks > (long long)per_sm * dev->sms) blocks = (long long)per_sm * dev->sms;
+  kern[slot]<<<(unsigned)blocks, 256, 0, st>>>(p);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? GQA_ATTN_OK : cuda_fail("launch(kv_append)", e, GQA_ATTN_ERR_LAUNCH);
 }

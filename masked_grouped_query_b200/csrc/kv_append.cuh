@@ -12,7 +12,7 @@
 // One thread moves 8 consecutive elements of one (batch, token, head) row,
 // so every 16- or 32-byte access is aligned and a warp covers whole rows:
 // the kernel is a strided copy, bound by HBM bandwidth (bytes read + bytes
-// written), with a grid-stride loop over a grid sized from the SM count and
+// written), with a grid-stride loop over one wave of resident blocks and
 // 32-bit index arithmetic.
 #pragma once
 

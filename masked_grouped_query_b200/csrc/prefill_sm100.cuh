@@ -36,9 +36,10 @@
 // The two softmax warpgroups work on their own tiles at the same time, out
 // of phase: while one computes its softmax the tensor core runs the other
 // tile's P.V and next S, and the two warps each SM sub-partition holds (one
-// per tile) hide each other's waits.  Of every 32 scores of a row, a fixed
-// share takes 2^x from a polynomial on the FMA pipe instead of the MUFU
-// unit, so the two pipes share the exponentials.
+// per tile) hide each other's waits.  The softmax code is one compact path
+// for every tile (masked tiles get -inf written over their hidden scores
+// first): separate unrolled copies for masked tiles missed the instruction
+// cache each time they ran.
 //
 // Fully masked key tiles are never loaded; tiles wholly inside every row's
 // visible range skip the per-element mask.  All waits are bounded.
@@ -64,8 +65,10 @@ constexpr int kRegsHigh = 208;
 constexpr int kRegSplitTotal = 4 * 32 * kRegsLow + 8 * 32 * kRegsHigh;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Of every 16 score pairs (32 keys) of a row, pairs [kEmuFrom, 16) take 2^x
-// from exp2_poly_x2 (FMA pipe) on tiles without a mask, the rest from MUFU.
-constexpr int kEmuFrom = 12;
+// from exp2_poly_x2 (FMA pipe), the rest from MUFU.  16: none (measured on
+// B200: offloading a quarter or a half to the FMA pipe was 3-8% slower;
+// the softmax here is not bound by the MUFU rate).
+constexpr int kEmuFrom = 16;
 
 struct PrefillParams {
   __nv_bfloat16* o;
@@ -458,14 +461,17 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           mma_commit(&s_full[t]);
           if (--s_left == 0) mma_commit(q_empty);  // Q no longer read: it may be reloaded
         };
+        // P.V: the V descriptor is built once; the K-steps advance its
+        // 14-bit address field by compile-time offsets (sdesc_advance).
         auto issue_pv_at = [&](int t, uint32_t vslot, bool first) {
           const uint32_t p_tmem = tmem + t * 128;
           const uint32_t o_tmem = tmem + 256 + t * 128;
+          const uint64_t vd = sdesc_sw128(vslot, C::kBoxBytes, 1024);
           tc_fence_after();
-          for (int ks = 0; ks < kPfN / 16; ++ks)
-            mma_bf16_ts(o_tmem, p_tmem + ks * 8,
-                        sdesc_sw128(vslot + ks * 2048, C::kBoxBytes, 1024), idesc_o,
-                        (!first || ks > 0) ? 1u : 0u);
+          mma_bf16_ts(o_tmem, p_tmem, vd, idesc_o, first ? 0u : 1u);
+#pragma unroll
+          for (int ks = 1; ks < kPfN / 16; ++ks)
+            mma_bf16_ts(o_tmem, p_tmem + ks * 8, sdesc_advance(vd, ks * 2048), idesc_o, 1u);
         };
         bool first_pv[2] = {true, true};
         if (it.paired) {
@@ -601,50 +607,52 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         ++n_s;
         if (!ok) break;
         tc_fence_after();
-        const int clo = lo - ktile0, chi = hi - ktile0;  // visible columns of this row
-        // Pass 1: the row's 128 scores, for its max (and, with a softcap, its
-        // min: when every |x / s| of the warp's rows is <= 1/2, tanh runs as
-        // an odd polynomial on the FMA pipe; the raw scores decide it).
+        // Visible columns of this row: c is hidden iff (unsigned)(c - vlo) >
+        // vspan (the range clamped to the tile; an empty range hides all).
+        const int clo = max(lo - ktile0, 0), chi = min(hi - ktile0, kPfN - 1);
+        const int vlo = chi >= clo ? clo : kPfN;
+        const unsigned vspan = chi >= clo ? (unsigned)(chi - clo) : 0u;
+        // Pass 1, 32 scores at a time: the row's max over its visible keys
+        // and, with a softcap, the raw scores' range (when every |x / s| of
+        // the warp's rows is <= 1/2, tanh runs as an odd polynomial on the
+        // FMA pipe).  On tiles with a mask the hidden scores become -inf and
+        // are written back, so pass 2 is the same code on every tile.
         bool small_y = false;
-        float mraw;
+        float mraw = -INFINITY;
         {
-          uint32_t sr[128];
-          tmem_ld128(s_tm, sr);
-          tmem_ld_wait();
-          auto xv = [&](int c) { return __uint_as_float(sr[c]); };
-          // Visible score, or -inf.
-          auto xm = [&](int c) { return c < clo || c > chi ? -INFINITY : xv(c); };
-          auto row_max = [&](auto score) {
-            float mx[4];
+          float amax = 0.f;  // max |x| over the raw scores (softcap check)
+#pragma unroll 1
+          for (int g = 0; g < 4; ++g) {
+            uint32_t sr[32];
+            tmem_ld32(s_tm + 32 * g, sr);
+            tmem_ld_wait();
+            if constexpr (kCap) {
+              float mx = fmaxf(__uint_as_float(sr[0]), __uint_as_float(sr[1]));
+              float mn = fminf(__uint_as_float(sr[0]), __uint_as_float(sr[1]));
 #pragma unroll
-            for (int k = 0; k < 4; ++k) mx[k] = fmaxf(score(2 * k), score(2 * k + 1));
-#pragma unroll
-            for (int c = 8; c < 128; c += 8)
-#pragma unroll
-              for (int k = 0; k < 4; ++k) mx[k] = fmax3(mx[k], score(c + 2 * k), score(c + 2 * k + 1));
-            return fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
-          };
-          if constexpr (kCap) {
-            float mx[4], mn[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              mx[k] = fmaxf(xv(2 * k), xv(2 * k + 1));
-              mn[k] = fminf(xv(2 * k), xv(2 * k + 1));
-            }
-#pragma unroll
-            for (int c = 8; c < 128; c += 8)
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                mx[k] = fmax3(mx[k], xv(c + 2 * k), xv(c + 2 * k + 1));
-                mn[k] = fmin3(mn[k], xv(c + 2 * k), xv(c + 2 * k + 1));
+              for (int c = 2; c < 32; c += 2) {
+                mx = fmax3(mx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+                mn = fmin3(mn, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
               }
-            mraw = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
-            const float mna = fmin3(mn[0], mn[1], fminf(mn[2], mn[3]));
-            small_y = __all_sync(0xffffffffu, fmaxf(mraw, -mna) * p.cap_in <= 0.5f);
-            if (need_mask) mraw = row_max(xm);
-          } else {
-            mraw = need_mask ? row_max(xm) : row_max(xv);
+              amax = fmax3(amax, mx, -mn);
+            }
+            if (need_mask) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                if ((unsigned)(32 * g + c - vlo) > vspan) sr[c] = __float_as_uint(-INFINITY);
+              tmem_st32(s_tm + 32 * g, sr);
+            }
+            float m2[2] = {fmaxf(__uint_as_float(sr[0]), __uint_as_float(sr[1])),
+                           fmaxf(__uint_as_float(sr[2]), __uint_as_float(sr[3]))};
+#pragma unroll
+            for (int c = 4; c < 32; c += 4) {
+              m2[0] = fmax3(m2[0], __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+              m2[1] = fmax3(m2[1], __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
+            }
+            mraw = fmax3(mraw, m2[0], m2[1]);
           }
+          if (need_mask) tmem_st_wait();  // pass 2 reads the masked scores
+          if constexpr (kCap) small_y = __all_sync(0xffffffffu, amax * p.cap_in <= 0.5f);
         }
         const float mt = mraw == -INFINITY ? -INFINITY
                          : kCap ? p.cap_out * tanh_fast(mraw * p.cap_in)
@@ -673,47 +681,45 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         const float base = m == -INFINITY ? 0.f : m;
         // Pass 2: p = 2^(logit - base) as bf16 pairs into TMEM over S, 32
-        // keys at a time: the scores of keys 32g .. 32g + 31 are read again
-        // (the next group's read is in flight while this one is computed) and
-        // their P lands in columns [16g, 16g + 16), all of whose scores were
-        // read before.  Pairs [kEmuFrom, 16) of each group take the FMA-pipe
-        // 2^x on tiles without a mask; a hidden key gives p = 0 (its logit is
-        // -inf, or it is zeroed explicitly).
+        // keys at a time (two groups per turn of a loop; the next group's
+        // read is in flight while one is computed): P of keys 32g .. 32g + 31
+        // lands in columns [16g, 16g + 16), whose scores were read before.
+        // Pairs [kEmuFrom, 16) of each group take the FMA-pipe 2^x.  A
+        // hidden key's score is -inf and gives p = 0; the logit transforms
+        // that do not carry -inf through (`explicit_hidden`) zero it by
+        // column range instead.
         f2 acc[4] = {0ull, 0ull, 0ull, 0ull};
-        auto emit = [&](auto logit2, auto emu, auto hidden) {
-          uint32_t buf[2][32];
-          tmem_ld32(s_tm, buf[0]);
-          tmem_ld_wait();
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            if (g < 3) tmem_ld32(s_tm + 32 * (g + 1), buf[(g + 1) & 1]);
-            const uint32_t(&sv)[32] = buf[g & 1];
+        auto emit = [&](auto logit2, auto explicit_hidden) {
+          constexpr bool kHid = decltype(explicit_hidden)::value;
+          auto group = [&](const uint32_t(&sv)[32], int g) {
             uint32_t pk[16];
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-              float xa = __uint_as_float(sv[2 * c]), xb = __uint_as_float(sv[2 * c + 1]);
-              const int col = 32 * g + 2 * c;
-              bool ha = false, hb = false;
-              if constexpr (decltype(hidden)::value) {
-                ha = col < clo || col > chi;
-                hb = col + 1 < clo || col + 1 > chi;
-                if constexpr (!kCap) {  // -inf logits give p = 0 by themselves
-                  if (ha) xa = -INFINITY;
-                  if (hb) xb = -INFINITY;
-                }
-              }
-              const f2 y = logit2(f2_pack(xa, xb));
-              f2 pv = (decltype(emu)::value && c >= kEmuFrom) ? exp2_poly_x2(y) : exp2_mufu_x2(y);
-              if constexpr (decltype(hidden)::value && kCap) {
+              const f2 y = logit2(f2_pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])));
+              f2 pv = c >= kEmuFrom ? exp2_poly_x2(y) : exp2_mufu_x2(y);
+              if constexpr (kHid) {
                 float a, b;
                 f2_unpack(pv, a, b);
-                pv = f2_pack(ha ? 0.f : a, hb ? 0.f : b);
+                const int col = 32 * g + 2 * c;
+                pv = f2_pack((unsigned)(col - vlo) > vspan ? 0.f : a,
+                             (unsigned)(col + 1 - vlo) > vspan ? 0.f : b);
               }
               acc[c & 3] = f2_add(acc[c & 3], pv);
               pk[c] = pack_bf16_f2(pv);
             }
             tmem_st16(s_tm + 16 * g, pk);
-            if (g < 3) tmem_ld_wait();
+          };
+          uint32_t b0[32], b1[32];
+          tmem_ld32(s_tm, b0);
+          tmem_ld_wait();
+#pragma unroll 1
+          for (int g = 0; g < 4; g += 2) {
+            tmem_ld32(s_tm + 32 * (g + 1), b1);
+            group(b0, g);
+            tmem_ld_wait();
+            if (g + 2 < 4) tmem_ld32(s_tm + 32 * (g + 2), b0);
+            group(b1, g + 1);
+            if (g + 2 < 4) tmem_ld_wait();
           }
         };
         using Yes = std::true_type;
@@ -721,45 +727,38 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const f2 nb = f2_pack(-base, -base);
         if constexpr (!kCap) {
           const f2 sc = f2_pack(p.logit_scale, p.logit_scale);
-          auto logit = [&](f2 v) { return f2_fma(v, sc, nb); };
-          if (need_mask) emit(logit, No(), Yes());
-          else emit(logit, Yes(), No());
+          emit([&](f2 v) { return f2_fma(v, sc, nb); }, No());
         } else if (small_y) {
           // cap_out * tanh(x * cap_in) = x * Q(x^2), the odd polynomial with
-          // cap_in^(2k+1) * cap_out folded into its coefficients.
+          // cap_in^(2k+1) * cap_out folded into its coefficients.  Degree 5:
+          // its top coefficient is positive, so x = -inf gives -inf.
           const float ci2 = p.cap_in * p.cap_in, cc = p.cap_out * p.cap_in;
           if constexpr (kCapDeg == 5) {
             const f2 q0 = f2_pack(cc * kTanh5C1, cc * kTanh5C1);
             const f2 q1 = f2_pack(cc * ci2 * kTanh5C3, cc * ci2 * kTanh5C3);
             const f2 q2 = f2_pack(cc * ci2 * ci2 * kTanh5C5, cc * ci2 * ci2 * kTanh5C5);
-            auto logit = [&](f2 v) {
+            emit([&](f2 v) {
               const f2 v2 = f2_mul(v, v);
               return f2_fma(v, f2_fma(f2_fma(q2, v2, q1), v2, q0), nb);
-            };
-            if (need_mask) emit(logit, No(), Yes());
-            else emit(logit, Yes(), No());
+            }, No());
           } else {
             const f2 q0 = f2_pack(cc * kTanhC1, cc * kTanhC1);
             const f2 q1 = f2_pack(cc * ci2 * kTanhC3, cc * ci2 * kTanhC3);
             const f2 q2 = f2_pack(cc * ci2 * ci2 * kTanhC5, cc * ci2 * ci2 * kTanhC5);
             const f2 q3 = f2_pack(cc * ci2 * ci2 * ci2 * kTanhC7, cc * ci2 * ci2 * ci2 * kTanhC7);
-            auto logit = [&](f2 v) {
+            emit([&](f2 v) {
               const f2 v2 = f2_mul(v, v);
               return f2_fma(v, f2_fma(f2_fma(f2_fma(q3, v2, q2), v2, q1), v2, q0), nb);
-            };
-            if (need_mask) emit(logit, No(), Yes());
-            else emit(logit, Yes(), No());
+            }, Yes());
           }
         } else {
-          // Large arguments (rare): the hardware tanh, every exponential on MUFU.
+          // Large arguments (rare): the hardware tanh, which maps -inf to -1.
           const float co = p.cap_out, ci = p.cap_in;
-          auto logit = [&](f2 v) {
+          emit([&](f2 v) {
             float a, b;
             f2_unpack(v, a, b);
             return f2_pack(fmaf(co, tanh_fast(a * ci), -base), fmaf(co, tanh_fast(b * ci), -base));
-          };
-          if (need_mask) emit(logit, No(), Yes());
-          else emit(logit, No(), No());
+          }, Yes());
         }
         {
           float a0, a1, b0, b1, c0, c1, d0, d1;
@@ -823,7 +822,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if constexpr (!kSplit) {
         if (ti.nrows > 0 && quarter * 32 < ti.nrows) {
           const bool have = act > 0;  // warp-uniform
-          const bool live = have && l > 0.f;
+          const bool live = have && m != -INFINITY && l > 0.f;
           const float inv = live ? 1.0f / l : 0.f;
           for (int c0 = 0; c0 < p.d_pad; c0 += 64)
             store_box(ti, c0, [&](int col, float (&v)[16]) {

@@ -276,6 +276,18 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[15])
       : "memory");
 }
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -291,6 +303,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   d |= (uint64_t)1u << 46;
   d |= (uint64_t)2u << 61;
   return d;
+}
+
+// The descriptor d with its start address advanced by `bytes` (a multiple of
+// 16): the 14-bit address field wraps like sdesc_sw128's own masking, so
+// no carry reaches the next field.
+__device__ __forceinline__ uint64_t sdesc_advance(uint64_t d, uint32_t bytes) {
+  const uint32_t lo = (uint32_t)d;
+  const uint32_t nlo = (lo & ~0x3FFFu) | ((lo + (bytes >> 4)) & 0x3FFFu);
+  return (d & 0xFFFFFFFF00000000ull) | nlo;
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 accumulate.
@@ -434,28 +455,30 @@ constexpr float kExp2C2 = 0.22606714069843292f;
 constexpr float kExp2C3 = 0.07802452892065048f;
 
 // 2^y for a pair of y <= 2^7 without the MUFU unit (Cody-Waite): y is
-// clamped to >= -126, split as y = j + f with j = floor(y) (the add of
+// clamped to >= -256, split as y = j + f with j = floor(y) (the add of
 // 1.5 * 2^23 rounded toward -inf leaves j in the low mantissa bits of the
 // sum) and f in [0, 1); the result is P(f) with j added to its exponent
-// field, which the clamp keeps >= 0.  Relative error 7.5e-5 for y >= -125;
-// below that the result is a non-negative value under 2^-124, not exactly
-// 2^y (callers use it only where such values are negligible next to the
-// row's largest term, 2^0 or more).
+// field as a signed integer (no overflow for j >= -256), and a negative
+// sum -- j < -127, or -inf -- becomes +0.  Relative error 7.5e-5 for
+// y >= -125; below that a non-negative value under 2^-124, exactly 0 for
+// y < -127 (as the hardware ex2 gives 0 for -inf).
 __device__ __forceinline__ f2 exp2_poly_x2(f2 y) {
   float a, b;
   f2_unpack(y, a, b);
-  const f2 yc = f2_pack(fmaxf(a, -126.f), fmaxf(b, -126.f));
+  const f2 yc = f2_pack(fmaxf(a, -256.f), fmaxf(b, -256.f));
   const f2 magic = f2_pack(12582912.f, 12582912.f);
   const f2 t = f2_add_rm(yc, magic);
   const f2 fr = f2_sub(yc, f2_sub(t, magic));
   f2 q = f2_fma(fr, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
   q = f2_fma(q, fr, f2_pack(kExp2C1, kExp2C1));
   q = f2_fma(q, fr, f2_pack(kExp2C0, kExp2C0));
-  uint32_t t0, t1, q0, q1;
+  int32_t t0, t1, q0, q1;
   asm("mov.b64 {%0, %1}, %2;" : "=r"(t0), "=r"(t1) : "l"(t));
   asm("mov.b64 {%0, %1}, %2;" : "=r"(q0), "=r"(q1) : "l"(q));
+  const int32_t r0 = max(q0 + (int32_t)((uint32_t)t0 << 23), 0);
+  const int32_t r1 = max(q1 + (int32_t)((uint32_t)t1 << 23), 0);
   f2 r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(q0 + (t0 << 23)), "r"(q1 + (t1 << 23)));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(r0), "r"(r1));
   return r;
 }
 
