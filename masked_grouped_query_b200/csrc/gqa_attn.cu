@@ -39,6 +39,7 @@ struct DeviceInfo {
   bool decode_attr[8] = {false, false, false, false, false, false, false, false};
   bool prefill_attr[12] = {};  // per (DCH, softcap degree, split) instantiation
   int append_blocks[4] = {};    // resident kv_append blocks per SM, per instantiation
+  bool append_runs_ready[4] = {};  // staged-runs kernel's smem attribute set
   // Clusters of n CTAs of a split instantiation that can be resident at once
   // (cudaOccupancyMaxActiveClusters); -1 = not asked yet.
   int cluster_max[12][9];
@@ -160,6 +161,9 @@ int cuda_fail(const char* where, cudaError_t e, int code) {
 inline long long ceil_div(long long a, long long b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Longest key split of the small-row-block decode plan, in key tiles.
+constexpr int kDecMaxSplitTiles = 128;
+
 int plan_decode(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
   pl->path = kPathDecode;
   pl->ks = pr.d <= 64 ? 4 : pr.d <= 128 ? 8 : pr.d <= 192 ? 12 : 16;
@@ -183,13 +187,19 @@ int plan_decode(const Problem& pr, const DeviceInfo& dev, Plan* pl) {
   } else if (forced > 0) {
     tps = forced;
   } else {
-    // Splits per row block, measured on B200 (L2 flushed): single-token
-    // blocks (keys-as-M variant, two CTAs per SM) do best with ~3.5 CTAs per
-    // SM in total; larger row blocks (one CTA per SM, partial traffic of 64
-    // rows per split) with about two thirds of a wave.
-    const double per_sm = pl->block_rows <= 8 ? 3.5 : 0.65;
+    // Splits per row block, measured on B200 (L2 flushed).  Small row
+    // blocks (keys-as-M variant): about one CTA per SM in total, since every
+    // extra split adds partial traffic and a merge at the end, but no split
+    // longer than kDecMaxSplitTiles tiles (long caches keep several splits per
+    // unit so that the grid still has a second CTA per SM to switch to).
+    // Larger row blocks (one CTA per SM, partial traffic of 64 rows per
+    // split): about two thirds of a wave.
+    const bool small = pl->block_rows <= 8;
+    const double per_sm = small ? 1.0 : 0.65;
     long long want = (long long)(per_sm * dev.sms / (double)base + 0.5);
     if (want < 1) want = 1;
+    if (small && want < ceil_div(max_tiles, kDecMaxSplitTiles))
+      want = ceil_div(max_tiles, kDecMaxSplitTiles);
     tps = (int)ceil_div(max_tiles, want);
     if (tps < 4) tps = 4;
   }
@@ -998,6 +1008,58 @@ static int append_checks(void* k_cache, void* v_cache, const void* new_k, const 
   return GQA_ATTN_OK;
 }
 
+// The staged-runs kernel applies when the source and the cache share their
+// layout (so one batch row, or one (batch, head) row, of new tokens is one
+// contiguous run in both), a ring does not wrap inside the block, and the
+// block is large enough for whole chunks to pay off (runs of at least 1024
+// elements, a million elements per tensor); small appends (a decode step)
+// keep the generic kernel.
+static bool append_runs_eligible(const KvAppendParams& p, long long n) {
+  if (p.cache_seq_major == p.new_head_major) return false;
+  const long long slot0 = p.ring ? (long long)p.position % p.slots : p.position;
+  if (slot0 + p.count > p.slots) return false;
+  const long long run_len =
+      p.cache_seq_major ? (long long)p.count * p.heads * p.head_dim : (long long)p.count * p.head_dim;
+  return run_len >= 1024 && n >= (1LL << 20);
+}
+
+static int launch_append_runs(const KvAppendParams& p, bool nf, bool cf, DeviceInfo* dev,
+                              cudaStream_t st) {
+  KvRunParams r;
+  r.k_cache = p.k_cache;
+  r.v_cache = p.v_cache;
+  r.new_k = p.new_k;
+  r.new_v = p.new_v;
+  const long long slot0 = p.ring ? (long long)p.position % p.slots : p.position;
+  const uint64_t row = p.cache_seq_major ? (uint64_t)p.heads * p.head_dim : (uint64_t)p.head_dim;
+  r.runs = p.cache_seq_major ? (uint32_t)p.batch : (uint32_t)(p.batch * p.heads);
+  r.run_len = (uint32_t)(p.count * row);
+  r.chunks_per_run = (r.run_len + kRunChunk - 1) / kRunChunk;
+  r.src_run_stride = r.run_len;
+  r.dst_run_stride = (uint64_t)p.slots * row;
+  r.dst_first = (uint64_t)slot0 * row;
+  const int slot = (nf ? 2 : 0) + (cf ? 1 : 0);
+  void (*const kern[4])(const KvRunParams) = {
+      kv_append_runs_kernel<false, false>, kv_append_runs_kernel<false, true>,
+      kv_append_runs_kernel<true, false>, kv_append_runs_kernel<true, true>};
+  const uint32_t smem = nf ? run_smem_bytes<true>() : run_smem_bytes<false>();
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!dev->append_runs_ready[slot]) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(kern[slot], cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return cuda_fail("kv_append smem attribute", e, GQA_ATTN_ERR_LAUNCH);
+      dev->append_runs_ready[slot] = true;
+    }
+  }
+  const long long items = 2LL * r.runs * r.chunks_per_run;
+  const long long cap = (long long)kRunCtasPerSm * dev->sms;
+  const long long blocks = items < cap ? items : cap;
+  kern[slot]<<<(unsigned)blocks, kRunThreads, smem, st>>>(r);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? GQA_ATTN_OK : cuda_fail("launch(kv_append runs)", e, GQA_ATTN_ERR_LAUNCH);
+}
+
 int gqa_attn_kv_append(void* k_cache, void* v_cache, const void* new_k, const void* new_v,
                        int batch, int cache_slots, int num_kv_heads, int head_dim, int position,
                        int count, unsigned int flags, int* new_length, void* stream) {
@@ -1028,6 +1090,7 @@ int gqa_attn_kv_append(void* k_cache, void* v_cache, const void* new_k, const vo
   const long long chunks = 2 * n / 8;  // 8 elements per thread, keys then values
   cudaStream_t st = (cudaStream_t)stream;
   const bool nf = !(flags & GQA_KV_NEW_BF16), cf = (flags & GQA_KV_CACHE_F32) != 0;
+  if (append_runs_eligible(p, n)) return launch_append_runs(p, nf, cf, dev, st);
   // One wave: as many blocks as are resident at once (the grid-stride loop
   // takes the rest), so no second partial wave trails the first.
   const int slot = (nf ? 2 : 0) + (cf ? 1 : 0);

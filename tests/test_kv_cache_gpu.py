@@ -93,6 +93,44 @@ def test_append_bit_exact(combo, shape):
     assert_same_bits(bits_of(from_layout(vc.cpu(), not seq_major)), want_v, "value cache")
 
 
+# Blocks large enough for the staged-runs kernel (a million new elements per
+# tensor, runs of at least 1024 elements, cache and tokens in the same
+# layout).  1030 tokens x 4 heads x 128: a (B, S, H, D) run is 128.75
+# chunks of 4096 elements and a (B, H, S, D) run 32.19, so every run ends in
+# a ragged chunk.  Ring positions: 4900 lands at slot 100 (no wrap, staged
+# kernel); 5000 lands at slot 200 and wraps (generic kernel).
+STAGED = [(cache_dt, new_dt, seq_major)
+          for cache_dt in (torch.bfloat16, torch.float32)
+          for new_dt in (torch.float32, torch.bfloat16)
+          for seq_major in (True, False)]
+
+
+@pytest.mark.parametrize("combo", STAGED, ids=[
+    f"{str(c[0])[6:]}-new_{str(c[1])[6:]}-{'seq' if c[2] else 'head'}" for c in STAGED])
+@pytest.mark.parametrize("where", [("linear", 100), ("ring", 4900), ("ring", 5000)])
+def test_append_large_blocks_bit_exact(combo, where):
+    cache_dt, new_dt, seq_major = combo
+    mode, pos = where
+    b, s, h, d, length = 2, 1200, 4, 128, 1030
+    x = make_cache_inputs(b, s, h, d, length, cache_dtype=cache_dt, new_dtype=new_dt,
+                          seed=7 + pos + d)
+    kc = to_layout(x["k_cache"], not seq_major).cuda()
+    vc = to_layout(x["v_cache"], not seq_major).cuda()
+    nk = to_layout(x["new_k"], not seq_major).cuda()
+    nv = to_layout(x["new_v"], not seq_major).cuda()
+    ring = mode == "ring"
+    n = mgq.kv_append(kc, vc, nk, nv, pos, seq_major=seq_major, new_head_major=not seq_major,
+                      ring=ring)
+    torch.cuda.synchronize()
+    update = okv.ring_update if ring else okv.kv_update
+    want_k, want_v, want_n = update(bits_of(x["k_cache"]), bits_of(x["v_cache"]),
+                                    bits_of(x["new_k"]), bits_of(x["new_v"]), pos)
+    assert n == want_n
+    assert_same_bits(bits_of(from_layout(kc.cpu(), not seq_major)), want_k, "key cache")
+    assert_same_bits(bits_of(from_layout(vc.cpu(), not seq_major)), want_v, "value cache")
+    assert mgq.status() == 0
+
+
 def test_append_page_examples():
     # The three worked examples printed on "KV Cache Update at a Position"
     # ("Examples": fp32 caches (B, S, H, D), fp32 new vectors), through the

@@ -32,8 +32,8 @@ def _call(fn, w, q, k, v, out):
 
 
 CASES = [
-    # decode, 4:1 GQA, several splits (partials ~2.6 MB)
-    Workload("c2like", 16, 1, 8192, 32, 8, 128, True, None, None, 41),
+    # decode, 4:1 GQA, 32 (batch, kv head) units: five key splits each
+    Workload("c2like", 4, 1, 8192, 32, 8, 128, True, None, None, 41),
     # multi-token 16:1 decode with window and softcap (partials ~4.5 MB)
     Workload("c5like", 2, 4, 8192, 64, 4, 128, True, 4096, 30.0, 42),
     # one split: no scratch used at all
