@@ -60,8 +60,8 @@ constexpr int kPfThreads = 32 * kPfWarps;
 // the two softmax warpgroups rise to kRegsHigh.  The host checks before every
 // launch that 4*32*kRegsLow + 8*32*kRegsHigh fits in the registers the block
 // is launched with, so the increase can always be granted.
-constexpr int kRegsLow = 88;
-constexpr int kRegsHigh = 208;
+constexpr int kRegsLow = 120;
+constexpr int kRegsHigh = 192;
 constexpr int kRegSplitTotal = 4 * 32 * kRegsLow + 8 * 32 * kRegsHigh;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 // Of every 16 score pairs (32 keys) of a row, pairs [kEmuFrom, 16) take 2^x
@@ -449,14 +449,20 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           return mbar_wait(&kv_full[u % C::kSlots], (u / C::kSlots) & 1, kStatusTimeoutMma);
         };
         auto release = [&](int idx) { mma_commit(&kv_empty[(ubase + idx) % C::kSlots]); };
+        // S: both descriptors are built once; the K-steps (ksteps <= 4 * DCH)
+        // advance their address fields by compile-time offsets.
         auto issue_s_at = [&](int t, uint32_t kslot) {
           const uint32_t qt = sq_addr + (it.paired ? 0 : t * C::kTileBytes);
           const uint32_t d_tmem = tmem + t * 128;
+          const uint64_t qd = sdesc_sw128(qt, 16, 1024);
+          const uint64_t kd = sdesc_sw128(kslot, 16, 1024);
           tc_fence_after();
-          for (int ks = 0; ks < ksteps; ++ks) {
+          mma_bf16_ss(d_tmem, qd, kd, idesc_s, 0u);
+#pragma unroll
+          for (int ks = 1; ks < 4 * DCH; ++ks) {
+            if (ks >= ksteps) break;
             const uint32_t off = (ks >> 2) * C::kBoxBytes + (ks & 3) * 32;
-            mma_bf16_ss(d_tmem, sdesc_sw128(qt + off, 16, 1024),
-                        sdesc_sw128(kslot + off, 16, 1024), idesc_s, ks > 0 ? 1u : 0u);
+            mma_bf16_ss(d_tmem, sdesc_advance(qd, off), sdesc_advance(kd, off), idesc_s, 1u);
           }
           mma_commit(&s_full[t]);
           if (--s_left == 0) mma_commit(q_empty);  // Q no longer read: it may be reloaded
