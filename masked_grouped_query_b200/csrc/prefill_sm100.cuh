@@ -64,11 +64,12 @@ constexpr int kRegsLow = 120;
 constexpr int kRegsHigh = 192;
 constexpr int kRegSplitTotal = 4 * 32 * kRegsLow + 8 * 32 * kRegsHigh;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
-// Of every 16 score pairs (32 keys) of a row, pairs [kEmuFrom, 16) take 2^x
-// from exp2_poly_x2 (FMA pipe), the rest from MUFU.  16: none (measured on
-// B200: offloading a quarter or a half to the FMA pipe was 3-8% slower;
-// the softmax here is not bound by the MUFU rate).
-constexpr int kEmuFrom = 16;
+// Without a softcap, pairs [kEmuFrom, 16) of every 16 score pairs (32 keys)
+// of a row take 2^x from exp2_poly_x2 (FMA pipe), the rest from MUFU.
+// Measured on B200: one pair in eight was 2-3% faster on the encoder shape;
+// a quarter or a half was slower.  The softcap kernels already spend FMA
+// work on the tanh polynomial and keep every 2^x on MUFU.
+constexpr int kEmuFrom = 14;
 
 struct PrefillParams {
   __nv_bfloat16* o;
@@ -112,8 +113,8 @@ struct PrefillCfg {
   static constexpr int kXchgOffset = 16384;
   static constexpr int kBarOffset = kQBytes + kRingBytes + kStageBytes;
   // q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2],
-  // drain, part_done[2], flag_ready[2]
-  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 1 + 2 + 2;
+  // drain, part_done[2], flag_ready[2], p_half[2]
+  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 1 + 2 + 2 + 2;
   static constexpr int kSmemBytes = 1024 + kBarOffset + kNumBars * 8 + 16;
 };
 
@@ -284,7 +285,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   // (flag_ready[t]).
   uint64_t* part_done = drain + 1;
   uint64_t* flag_ready = part_done + 2;
-  uint32_t* tmem_slot = (uint32_t*)(flag_ready + 2);
+  uint64_t* p_half = flag_ready + 2;  // [t]: P of keys 0..63 of tile t is in TMEM
+  uint32_t* tmem_slot = (uint32_t*)(p_half + 2);
   int* merge_flag = (int*)(tmem_slot + 1);  // [2]: 1 merge, 0 not the last, -1 wait gave up
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -300,6 +302,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 4);  // one arrival per warp of the tile's warpgroup
+      mbar_init(&p_half[t], 4);
       mbar_init(&o_done[t], 1);
     }
     mbar_init(drain, 1);
@@ -469,15 +472,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         };
         // P.V: the V descriptor is built once; the K-steps advance its
         // 14-bit address field by compile-time offsets (sdesc_advance).
-        auto issue_pv_at = [&](int t, uint32_t vslot, bool first) {
+        // Half h of P.V: keys 64h .. 64h + 63 (K-steps 4h .. 4h + 3).
+        auto issue_pv_half = [&](int t, uint32_t vslot, bool first, int h) {
           const uint32_t p_tmem = tmem + t * 128;
           const uint32_t o_tmem = tmem + 256 + t * 128;
           const uint64_t vd = sdesc_sw128(vslot, C::kBoxBytes, 1024);
           tc_fence_after();
-          mma_bf16_ts(o_tmem, p_tmem, vd, idesc_o, first ? 0u : 1u);
 #pragma unroll
-          for (int ks = 1; ks < kPfN / 16; ++ks)
-            mma_bf16_ts(o_tmem, p_tmem + ks * 8, sdesc_advance(vd, ks * 2048), idesc_o, 1u);
+          for (int k = 0; k < kPfN / 32; ++k) {
+            const int ks = h * (kPfN / 32) + k;
+            mma_bf16_ts(o_tmem, p_tmem + ks * 8, sdesc_advance(vd, ks * 2048), idesc_o,
+                        (first && ks == 0) ? 0u : 1u);
+          }
+        };
+        // P.V in two halves: the first as soon as the softmax has written
+        // P of keys 0..63 (p_half), the second after the whole tile (p_full).
+        auto issue_pv_at = [&](int t, uint32_t vslot, bool first, int nph) -> bool {
+          if (!mbar_wait(&p_half[t], nph & 1, kStatusTimeoutMma)) return false;
+          issue_pv_half(t, vslot, first, 0);
+          if (!mbar_wait(&p_full[t], nph & 1, kStatusTimeoutMma)) return false;
+          issue_pv_half(t, vslot, false, 1);
+          return true;
         };
         bool first_pv[2] = {true, true};
         if (it.paired) {
@@ -504,8 +519,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int t = 0; t < 2 && ok; ++t) {
               if (!tile_active(it, t, j)) continue;
               if (!(ok = pwait(1, up(t, j)))) break;  // V_t(j)
-              if (!(ok = mbar_wait(&p_full[t], n_act[t] & 1, kStatusTimeoutMma))) break;
-              issue_pv_at(t, paddr(1, up(t, j)), first_pv[t]);
+              if (!(ok = issue_pv_at(t, paddr(1, up(t, j)), first_pv[t], n_act[t]))) break;
               first_pv[t] = false;
               ++n_act[t];
               if (j == last_j[t]) mma_commit(&o_done[t]);
@@ -524,7 +538,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
         auto issue_s = [&](int t, int j) { issue_s_at(t, slot_addr(2 * j)); };
         auto issue_pv = [&](int t, int j, bool first) {
-          issue_pv_at(t, slot_addr(2 * j + 1), first);
+          return issue_pv_at(t, slot_addr(2 * j + 1), first, n_act[t]);
         };
 
         // Prologue: S(0) of both tiles (K_0's only readers, so its slot is
@@ -538,8 +552,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           bool k_next_ready = j + 1 >= it.j_count;
           for (int t = 0; t < 2 && ok; ++t) {
             if (tile_active(it, t, j)) {
-              if (!(ok = mbar_wait(&p_full[t], n_act[t] & 1, kStatusTimeoutMma))) break;
-              issue_pv(t, j, first_pv[t]);
+              if (!(ok = issue_pv(t, j, first_pv[t]))) break;
               first_pv[t] = false;
               ++n_act[t];
               if (j == last_j[t]) mma_commit(&o_done[t]);
@@ -702,7 +715,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
               const f2 y = logit2(f2_pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1])));
-              f2 pv = c >= kEmuFrom ? exp2_poly_x2(y) : exp2_mufu_x2(y);
+              f2 pv = (!kCap && c >= kEmuFrom) ? exp2_poly_x2(y) : exp2_mufu_x2(y);
               if constexpr (kHid) {
                 float a, b;
                 f2_unpack(pv, a, b);
@@ -726,6 +739,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             if (g + 2 < 4) tmem_ld32(s_tm + 32 * (g + 2), b0);
             group(b1, g + 1);
             if (g + 2 < 4) tmem_ld_wait();
+            if (g == 0) {  // P of keys 0..63 written: the first half of P.V may start
+              tmem_st_wait();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&p_half[t]);
+            }
           }
         };
         using Yes = std::true_type;
