@@ -148,7 +148,10 @@ int gqa_attn_describe(int batch, int q_len, int kv_len, int num_q_heads, int num
  * key 4: how those splits merge (0 = automatic: through distributed shared
  *        memory in one thread-block cluster per unit when a unit has 2 to 8
  *        CTAs and the whole grid fits on the device at once; -1 = always
- *        through the workspace).
+ *        through the workspace);
+ * key 5: 1 = the tcgen05 kernel's softcap path always finds the row max
+ *        before the exponentials (0 = automatic: caps up to about 63.8 use a
+ *        fixed exponent base and a single pass over the scores).
  * A forced path that cannot run these sizes falls back to automatic.
  * Returns GQA_ATTN_OK or GQA_ATTN_ERR_ARG for an unknown key.
  */

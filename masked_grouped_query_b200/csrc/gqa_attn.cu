@@ -56,6 +56,7 @@ std::atomic<int> g_force_path{0};
 std::atomic<int> g_no_cluster{0};
 std::atomic<int> g_force_tps{0};
 std::atomic<int> g_force_pf_splits{0};
+std::atomic<int> g_force_two_pass{0};  // 1: softcap kernels always take the row max first
 
 int device_info(DeviceInfo** out) {
   int dev = 0;
@@ -627,6 +628,12 @@ int launch_prefill_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, int csi
   p.logit_scale = kLog2e * rs;
   p.cap_in = kCap ? rs / pr.softcap : 0.f;
   p.cap_out = kCap ? pr.softcap * kLog2e : 0.f;
+  {
+    // Fixed exponent base for the degree-5 softcap path (see PrefillParams).
+    const float b = std::max(16.0f, 2.0f * p.cap_out - 120.0f);
+    p.cap_fixed = (kCapDeg == 5 && b <= 64.0f && g_force_two_pass.load() == 0) ? 1 : 0;
+    p.cap_base = p.cap_out - b;
+  }
   if (p.cluster_merge > 0) {
     // One item per CTA, clusters of csize consecutive CTAs (one unit each).
     cudaLaunchConfig_t cfg = {};
@@ -862,6 +869,10 @@ int gqa_attn_set_override(int key, int value) {
   }
   if (key == 4) {
     g_no_cluster.store(value < 0 ? 1 : 0);
+    return GQA_ATTN_OK;
+  }
+  if (key == 5) {
+    g_force_two_pass.store(value ? 1 : 0);
     return GQA_ATTN_OK;
   }
   return GQA_ATTN_ERR_ARG;

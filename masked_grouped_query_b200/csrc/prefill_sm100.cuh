@@ -89,6 +89,13 @@ struct PrefillParams {
                          // shared memory instead of the workspace; 0 = workspace merge
   int causal, window;
   float logit_scale, cap_in, cap_out;
+  // Softcap with a fixed exponent base (cap_fixed = 1): the capped logits,
+  // in log2 units, lie in [-cap_out, cap_out], so p = 2^(y - cap_base) with
+  // cap_base = cap_out - B stays in [2^(B - 2 cap_out), 2^B].  The host picks
+  // B = max(16, 2 cap_out - 120) and sets cap_fixed only when B <= 64, so p
+  // never overflows or leaves the normal range and no row max is needed.
+  int cap_fixed;
+  float cap_base;
   // Split partials (splits > 1): per (pair, tile, split) O as fp32
   // [d / 4][128 rows][4] (a thread moves four columns of its row as one
   // 16-byte access and a warp's accesses coalesce) and (m, l) per row;
@@ -636,6 +643,96 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // the warp's rows is <= 1/2, tanh runs as an odd polynomial on the
         // FMA pipe).  On tiles with a mask the hidden scores become -inf and
         // are written back, so pass 2 is the same code on every tile.
+        if constexpr (kCapDeg == 5) {
+          if (p.cap_fixed) {
+            // One pass over the scores, no row max: y = cap(x) - cap_base.
+            // Per 32-key group, the warp takes the degree-5 polynomial when
+            // every |x * cap_in| <= 1/2 (hidden keys as -inf then give p = 0),
+            // else the hardware tanh with hidden keys zeroed by column.
+            const float base = p.cap_base;
+            m = base;
+            const f2 nb = f2_pack(-base, -base);
+            const float ci2 = p.cap_in * p.cap_in, cc = p.cap_out * p.cap_in;
+            const f2 q0 = f2_pack(cc * kTanh5C1, cc * kTanh5C1);
+            const f2 q1 = f2_pack(cc * ci2 * kTanh5C3, cc * ci2 * kTanh5C3);
+            const f2 q2 = f2_pack(cc * ci2 * ci2 * kTanh5C5, cc * ci2 * ci2 * kTanh5C5);
+            f2 acc[4] = {0ull, 0ull, 0ull, 0ull};
+            auto group = [&](uint32_t(&sv)[32], int g) {
+              float mx = fmaxf(__uint_as_float(sv[0]), __uint_as_float(sv[1]));
+              float mn = fminf(__uint_as_float(sv[0]), __uint_as_float(sv[1]));
+#pragma unroll
+              for (int c = 2; c < 32; c += 2) {
+                mx = fmax3(mx, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
+                mn = fmin3(mn, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
+              }
+              const bool poly = __all_sync(0xffffffffu, fmaxf(mx, -mn) * p.cap_in <= 0.5f);
+              if (need_mask) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                  if ((unsigned)(32 * g + c - vlo) > vspan) sv[c] = __float_as_uint(-INFINITY);
+              }
+              uint32_t pk[16];
+              if (poly) {
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                  const f2 v = f2_pack(__uint_as_float(sv[2 * c]), __uint_as_float(sv[2 * c + 1]));
+                  const f2 v2 = f2_mul(v, v);
+                  const f2 pv = exp2_mufu_x2(f2_fma(v, f2_fma(f2_fma(q2, v2, q1), v2, q0), nb));
+                  acc[c & 3] = f2_add(acc[c & 3], pv);
+                  pk[c] = pack_bf16_f2(pv);
+                }
+              } else {
+                const float co = p.cap_out, ci = p.cap_in;
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                  const float a = __uint_as_float(sv[2 * c]), b = __uint_as_float(sv[2 * c + 1]);
+                  f2 pv = exp2_mufu_x2(f2_pack(fmaf(co, tanh_fast(a * ci), -base),
+                                               fmaf(co, tanh_fast(b * ci), -base)));
+                  if (need_mask) {
+                    float pa, pb;
+                    f2_unpack(pv, pa, pb);
+                    const int col = 32 * g + 2 * c;
+                    pv = f2_pack((unsigned)(col - vlo) > vspan ? 0.f : pa,
+                                 (unsigned)(col + 1 - vlo) > vspan ? 0.f : pb);
+                  }
+                  acc[c & 3] = f2_add(acc[c & 3], pv);
+                  pk[c] = pack_bf16_f2(pv);
+                }
+              }
+              tmem_st16(s_tm + 16 * g, pk);
+            };
+            uint32_t b0[32], b1[32];
+            tmem_ld32(s_tm, b0);
+            tmem_ld_wait();
+#pragma unroll 1
+            for (int g = 0; g < 4; g += 2) {
+              tmem_ld32(s_tm + 32 * (g + 1), b1);
+              group(b0, g);
+              tmem_ld_wait();
+              if (g + 2 < 4) tmem_ld32(s_tm + 32 * (g + 2), b0);
+              group(b1, g + 1);
+              if (g + 2 < 4) tmem_ld_wait();
+              if (g == 0) {  // P of keys 0..63 written: the first half of P.V may start
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_half[t]);
+              }
+            }
+            float a0, a1, c0, c1, d0, d1, e0, e1;
+            f2_unpack(acc[0], a0, a1);
+            f2_unpack(acc[1], c0, c1);
+            f2_unpack(acc[2], d0, d1);
+            f2_unpack(acc[3], e0, e1);
+            l += ((a0 + a1) + (c0 + c1)) + ((d0 + d1) + (e0 + e1));
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[t]);
+            ++act;
+            continue;
+          }
+        }
         bool small_y = false;
         float mraw = -INFINITY;
         {
@@ -802,6 +899,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // Paired items (every item of a launch, or none): the two warpgroups
       // meet at a named barrier below, so a warpgroup that gave up on a wait
       // still goes there (with ok = false) instead of leaving at once.
+      // Fixed-base softcap: a row without a visible key keeps m = -inf.
+      if constexpr (kCapDeg == 5)
+        if (p.cap_fixed && !(l > 0.f)) m = -INFINITY;
       const bool pair_x = kSplit && it.paired;
       if (!ok && !pair_x) break;
       // ---- epilogue.  The next item's first P.V of this tile may overwrite

@@ -103,6 +103,25 @@ def test_wide_logit_range_without_softcap(cfg):
     check_workload(Workload("wide", b, lq, lk, hq, hkv, d, False, None, None, lq + d), q_scale=30.0)
 
 
+@pytest.mark.parametrize("two_pass", [0, 1])
+@pytest.mark.parametrize("cap,q_scale", [(5.0, 1.0), (50.0, 1.0), (50.0, 20.0), (63.0, 3.0),
+                                         (64.0, 3.0), (200.0, 20.0)])
+def test_softcap_fixed_base_and_row_max_paths_agree(cap, q_scale, two_pass):
+    # Caps up to about 63.8 take one pass with a fixed exponent base (no row
+    # max); larger caps, and every cap with the override set, find the row
+    # max first.  Both must match the oracle on masked, ragged tiles, with
+    # logits inside the polynomial's range (q_scale 1) and saturating ones
+    # (q_scale 20, the hardware tanh).
+    mgq.set_override("softcap_two_pass", two_pass)
+    try:
+        for w in (Workload("fb", 1, 300, 700, 8, 2, 128, True, 256, cap, 7),
+                  Workload("fb2", 2, 129, 129, 4, 4, 72, False, None, cap, 8),
+                  Workload("fb3", 1, 4, 3000, 64, 4, 128, True, 1000, cap, 9)):
+            check_workload(w, q_scale=q_scale)
+    finally:
+        mgq.set_override("softcap_two_pass", 0)
+
+
 def test_zero_kv_len_gives_zeros():
     q = torch.randn(2, 4, 3, 64, device="cuda").bfloat16()
     k = torch.empty(2, 2, 0, 64, device="cuda", dtype=torch.bfloat16)
