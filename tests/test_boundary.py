@@ -129,12 +129,14 @@ def test_ring_rejects_bad_arguments_without_a_device(lib):
 
 
 def test_override_keys(lib):
-    # Keys 1-4 are knobs (host state only, no device needed); others are rejected.
-    for key in (1, 2, 3, 4):
+    # Keys 1-5 are knobs (host state only, no device needed); others are rejected.
+    for key in (1, 2, 3, 4, 5):
         assert lib.gqa_attn_set_override(key, 0) == 0
     assert lib.gqa_attn_set_override(4, -1) == 0
     assert lib.gqa_attn_set_override(4, 0) == 0
-    assert lib.gqa_attn_set_override(5, 0) == -12  # GQA_ATTN_ERR_ARG
+    assert lib.gqa_attn_set_override(5, 1) == 0
+    assert lib.gqa_attn_set_override(5, 0) == 0
+    assert lib.gqa_attn_set_override(6, 0) == -12  # GQA_ATTN_ERR_ARG
     assert lib.gqa_attn_set_override(0, 0) == -12
     with pytest.raises(KeyError):
         mgq.set_override("no_such_knob", 1)
