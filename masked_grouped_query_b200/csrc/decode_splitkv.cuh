@@ -60,13 +60,16 @@ struct DecodeParams {
   unsigned int* tickets;  // [unit][rb], zero between calls
 };
 
-template <int KS>
+// kDeep: a 5-stage ring (160 KB in flight for KS = 8) for grids of at most
+// one CTA per SM, where the 3-stage ring of two co-resident CTAs would leave
+// each SM with half the bytes in flight.
+template <int KS, bool kDeep = false>
 struct DecodeCfg {
   static constexpr int kDChunks = KS / 4;                 // 64-column TMA boxes
   static constexpr int kBoxBytes = kDecTile * 128;        // one 64-key x 64-col box
   static constexpr int kTileBytes = kDChunks * kBoxBytes; // K (or V) tile
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kStages = KS <= 8 ? 3 : 2;
+  static constexpr int kStages = kDeep ? 5 : KS <= 8 ? 3 : 2;
   static constexpr int kRingBytes = kStages * kStageBytes;
   static constexpr int kMergeBytes = kDecComputeWarps * 16 * (KS * 16 + 2) * 4;
   static constexpr int kSmemBytes =
@@ -79,11 +82,11 @@ struct DecodeCfg {
 // rows), with P^T moved into the B-operand layout by movmatrix -- so the
 // padded rows cost half as much as in the rows-as-M form and the O
 // accumulator needs half the registers (two CTAs per SM).
-template <int KS, bool kT>
+template <int KS, bool kT, bool kDeep = false>
 __global__ void __maxnreg__(kT ? 128 : 255)
     decode_splitkv_kernel(const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
-  using C = DecodeCfg<KS>;
+  using C = DecodeCfg<KS, kDeep>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
   uint8_t* ring = smem;

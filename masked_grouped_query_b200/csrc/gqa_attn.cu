@@ -36,7 +36,7 @@ struct DeviceInfo {
   bool probed = false;
   int sms = 0, major = 0, minor = 0;
   int smem_optin = 0;
-  bool decode_attr[8] = {false, false, false, false, false, false, false, false};
+  bool decode_attr[10] = {};  // per instantiation: [0, 8) 3/2-stage, [8, 10) 5-stage
   bool prefill_attr[12] = {};  // per (DCH, softcap degree, split) instantiation
   int append_blocks[4] = {};    // resident kv_append blocks per SM, per instantiation
   bool append_runs_ready[4] = {};  // staged-runs kernel's smem attribute set
@@ -417,19 +417,19 @@ int encode_map(CUtensorMap* map, const void* base, int cols, long long rows, lon
 }
 
 // ------------------------------------------------------------------ launches
-template <int KS, bool kT>
+template <int KS, bool kT, bool kDeep = false>
 int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void* q,
                      const void* k, const void* v, void* o, void* ws, void* tickets,
                      cudaStream_t stream) {
-  using C = DecodeCfg<KS>;
-  const int slot = (KS / 4 - 1) + (kT ? 4 : 0);
+  using C = DecodeCfg<KS, kDeep>;
+  const int slot = kDeep ? 8 + (KS / 4 - 1) : (KS / 4 - 1) + (kT ? 4 : 0);
   std::unique_lock<std::mutex> lk(g_mu);
   if (!dev.decode_attr[slot]) {
-    cudaError_t e = cudaFuncSetAttribute(decode_splitkv_kernel<KS, kT>,
+    cudaError_t e = cudaFuncSetAttribute(decode_splitkv_kernel<KS, kT, kDeep>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_splitkv_kernel<KS, kT>,
+      e = cudaFuncSetAttribute(decode_splitkv_kernel<KS, kT, kDeep>,
                                cudaFuncAttributePreferredSharedMemoryCarveout,
                                cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return cuda_fail("cudaFuncSetAttribute(decode)", e, GQA_ATTN_ERR_LAUNCH);
@@ -476,7 +476,7 @@ int launch_decode_ks(const Problem& pr, const Plan& pl, DeviceInfo& dev, const v
   p.part_o = (float*)ws;
   p.part_lse = ws ? (float*)((char*)ws + pl.off_lse) : nullptr;
   p.tickets = (unsigned int*)tickets;
-  decode_splitkv_kernel<KS, kT>
+  decode_splitkv_kernel<KS, kT, kDeep>
       <<<dim3((unsigned)pl.ctas), kDecThreads, C::kSmemBytes, stream>>>(tk, tv, p);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? GQA_ATTN_OK : cuda_fail("launch(decode)", e, GQA_ATTN_ERR_LAUNCH);
@@ -486,9 +486,15 @@ int launch_decode(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void
                   const void* k, const void* v, void* o, void* ws, void* tickets,
                   cudaStream_t stream) {
   if (pl.block_rows <= 8) {  // single-token decode shapes: keys-as-M variant
+    // At most one CTA per SM: the deeper ring keeps more bytes in flight.
+    const bool deep = pl.ctas <= dev.sms;
     switch (pl.ks) {
-      case 4: return launch_decode_ks<4, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
-      case 8: return launch_decode_ks<8, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+      case 4:
+        return deep ? launch_decode_ks<4, true, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
+                    : launch_decode_ks<4, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
+      case 8:
+        return deep ? launch_decode_ks<8, true, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream)
+                    : launch_decode_ks<8, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
       case 12: return launch_decode_ks<12, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
       default: return launch_decode_ks<16, true>(pr, pl, dev, q, k, v, o, ws, tickets, stream);
     }
