@@ -9,7 +9,8 @@
 //
 // Per CTA: one loader warp streams 64-key K and V tiles with TMA
 // (cp.async.bulk.tensor, 128-byte swizzle) into a ring of 3 stages (2 for
-// head_dim above 128) guarded by mbarriers;
+// head_dim above 128; 5 when the grid has at most one CTA per SM, see
+// DecodeCfg) guarded by mbarriers;
 // four compute warps run S = Q K^T and O += P V on the tensor cores with
 // mma.sync m16n8k16 (bf16 in, fp32 accumulate) and an online fp32 softmax
 // with the softcap and mask fused in.  Chunks end with a log-sum-exp partial

@@ -32,14 +32,21 @@
 //               mask, keeps the running max and sum in fp32 (online softmax,
 //               rescaling its O row in TMEM only when the max grows by more
 //               than 2^8), writes P as bf16 back over S in TMEM, and at the
-//               end of the item normalises its O row and stores it.
+//               end of the item normalises its O row and stores it.  P.V is
+//               handed over in two halves: keys 0..63 (p_half) while the
+//               softmax still works on keys 64..127 (p_full).  With a
+//               softcap the logits are bounded, so caps up to about 63.8 use
+//               a fixed exponent base and one pass over the scores, with no
+//               row max and no rescale (PrefillParams::cap_fixed).
 // The two softmax warpgroups work on their own tiles at the same time, out
 // of phase: while one computes its softmax the tensor core runs the other
 // tile's P.V and next S, and the two warps each SM sub-partition holds (one
-// per tile) hide each other's waits.  The softmax code is one compact path
-// for every tile (masked tiles get -inf written over their hidden scores
-// first): separate unrolled copies for masked tiles missed the instruction
-// cache each time they ran.
+// per tile) hide each other's waits.  The MMA thread serves tile A, then
+// tile B, which keeps them half a step apart; serving events as they come,
+// or making the warpgroups take turns, was measured slower.  The softmax
+// code is one compact path for every tile (masked tiles get -inf written
+// over their hidden scores first): separate unrolled copies for masked
+// tiles missed the instruction cache each time they ran.
 //
 // Fully masked key tiles are never loaded; tiles wholly inside every row's
 // visible range skip the per-element mask.  All waits are bounded.
