@@ -199,6 +199,25 @@ def test_deterministic(name):
     assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("shape,splits", [
+    ((16, 1, 8192, 32, 8, 128), 1),    # 128 units: one CTA per unit
+    ((4, 1, 8192, 32, 8, 128), 5),     # 32 units: about one CTA per SM in total
+    ((16, 1, 32768, 32, 8, 128), 4),   # no split longer than 128 key tiles
+])
+def test_decode_split_rule(shape, splits):
+    # Single-token decode plans aim at about one CTA per SM (148 SMs on B200),
+    # with no split longer than 128 key tiles of 64 keys.
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    plan = mgq.describe(*shape, True)
+    assert plan["path"] == "decode"
+    if sms == 148:
+        assert plan["splits"] == splits, plan
+    units = shape[0] * shape[4]
+    assert plan["ctas"] == units * plan["splits"]
+    assert -(-plan["tiles"] // plan["splits"]) <= 128 or plan["splits"] == 1
+
+
 @pytest.mark.parametrize("tps", [1, 3, 7, 1000])
 def test_forced_split_geometries_agree_with_oracle(tps):
     # The split-KV decode kernel, forced, at several split sizes.
