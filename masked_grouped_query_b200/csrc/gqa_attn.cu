@@ -1029,15 +1029,16 @@ static int append_checks(void* k_cache, void* v_cache, const void* new_k, const 
 // layout (so one batch row, or one (batch, head) row, of new tokens is one
 // contiguous run in both), a ring does not wrap inside the block, and the
 // block is large enough for whole chunks to pay off (runs of at least 1024
-// elements, a million elements per tensor); small appends (a decode step)
-// keep the generic kernel.
+// elements, a million elements per tensor) but its runs stay below 2^31
+// elements; small appends (a decode step) keep the generic kernel.
 static bool append_runs_eligible(const KvAppendParams& p, long long n) {
   if (p.cache_seq_major == p.new_head_major) return false;
   const long long slot0 = p.ring ? (long long)p.position % p.slots : p.position;
   if (slot0 + p.count > p.slots) return false;
   const long long run_len =
       p.cache_seq_major ? (long long)p.count * p.heads * p.head_dim : (long long)p.count * p.head_dim;
-  return run_len >= 1024 && n >= (1LL << 20);
+  // Run lengths and chunk offsets are 32-bit in the kernel.
+  return run_len >= 1024 && run_len < (1LL << 31) && n >= (1LL << 20);
 }
 
 static int launch_append_runs(const KvAppendParams& p, bool nf, bool cf, DeviceInfo* dev,
