@@ -37,12 +37,12 @@ struct DeviceInfo {
   int sms = 0, major = 0, minor = 0;
   int smem_optin = 0;
   bool decode_attr[10] = {};  // per instantiation: [0, 8) 3/2-stage, [8, 10) 5-stage
-  bool prefill_attr[12] = {};  // per (DCH, softcap degree, split) instantiation
+  bool prefill_attr[16] = {};  // per (DCH, softcap code, split) instantiation
   int append_blocks[4] = {};    // resident kv_append blocks per SM, per instantiation
   bool append_runs_ready[4] = {};  // staged-runs kernel's smem attribute set
   // Clusters of n CTAs of a split instantiation that can be resident at once
   // (cudaOccupancyMaxActiveClusters); -1 = not asked yet.
-  int cluster_max[12][9];
+  int cluster_max[16][9];
   DeviceInfo() {
     for (auto& a : cluster_max)
       for (int& n : a) n = -1;
@@ -507,15 +507,26 @@ int launch_decode(const Problem& pr, const Plan& pl, DeviceInfo& dev, const void
   }
 }
 
-// Softcap degree of the tcgen05 kernel's tanh polynomial: caps up to
-// kTanh5MaxCap take degree 5, larger caps degree 7, 0 = no softcap.
+// Exponent-base offset B of the fixed-base softcap path for this cap (in
+// log2 units, cap_out = softcap * log2 e): B = max(16, 2 cap_out - 120), used
+// only when B <= 64 (see PrefillParams::cap_fixed).
+float cap_base_offset(float cap_out) { return std::max(16.0f, 2.0f * cap_out - 120.0f); }
+
+// Softcap code of the tcgen05 kernel: 0 = no softcap; 3 = the degree-5
+// tanh polynomial with a fixed exponent base (no row max; caps up to about
+// 63.8); 5 = the degree-5 polynomial with the row max (caps up to
+// kTanh5MaxCap, or any cap when override key 5 asks for it); 7 = degree 7.
 int cap_degree(const Problem& pr) {
-  return pr.softcap > 0.f ? (pr.softcap <= kTanh5MaxCap ? 5 : 7) : 0;
+  if (!(pr.softcap > 0.f)) return 0;
+  if (pr.softcap > kTanh5MaxCap) return 7;
+  const bool fixed = cap_base_offset(pr.softcap * kLog2e) <= 64.0f && g_force_two_pass.load() == 0;
+  return fixed ? 3 : 5;
 }
 
 template <int DCH, int kCapDeg, bool kSplit>
 constexpr int prefill_slot() {
-  return (DCH - 1) + (kCapDeg == 5 ? 2 : kCapDeg == 7 ? 4 : 0) + (kSplit ? 6 : 0);
+  return (DCH - 1) + 2 * (kCapDeg == 5 ? 1 : kCapDeg == 7 ? 2 : kCapDeg == 3 ? 3 : 0) +
+         (kSplit ? 8 : 0);
 }
 
 // One-time per device and instantiation (under g_mu): the register-split
@@ -587,10 +598,12 @@ int prefill_cluster_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, int* c
 int prefill_cluster(const Problem& pr, const Plan& pl, DeviceInfo& dev, int* csize) {
   const int deg = cap_degree(pr);
   if (pl.dch == 1)
-    return deg == 5 ? prefill_cluster_k<1, 5>(pr, pl, dev, csize)
+    return deg == 3 ? prefill_cluster_k<1, 3>(pr, pl, dev, csize)
+         : deg == 5 ? prefill_cluster_k<1, 5>(pr, pl, dev, csize)
          : deg == 7 ? prefill_cluster_k<1, 7>(pr, pl, dev, csize)
                     : prefill_cluster_k<1, 0>(pr, pl, dev, csize);
-  return deg == 5 ? prefill_cluster_k<2, 5>(pr, pl, dev, csize)
+  return deg == 3 ? prefill_cluster_k<2, 3>(pr, pl, dev, csize)
+       : deg == 5 ? prefill_cluster_k<2, 5>(pr, pl, dev, csize)
        : deg == 7 ? prefill_cluster_k<2, 7>(pr, pl, dev, csize)
                   : prefill_cluster_k<2, 0>(pr, pl, dev, csize);
 }
@@ -634,12 +647,9 @@ int launch_prefill_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, int csi
   p.logit_scale = kLog2e * rs;
   p.cap_in = kCap ? rs / pr.softcap : 0.f;
   p.cap_out = kCap ? pr.softcap * kLog2e : 0.f;
-  {
-    // Fixed exponent base for the degree-5 softcap path (see PrefillParams).
-    const float b = std::max(16.0f, 2.0f * p.cap_out - 120.0f);
-    p.cap_fixed = (kCapDeg == 5 && b <= 64.0f && g_force_two_pass.load() == 0) ? 1 : 0;
-    p.cap_base = p.cap_out - b;
-  }
+  // Fixed exponent base (softcap code 3, see PrefillParams and cap_degree).
+  p.cap_fixed = kCapDeg == 3 ? 1 : 0;
+  p.cap_base = kCapDeg == 3 ? p.cap_out - cap_base_offset(p.cap_out) : 0.f;
   if (p.cluster_merge > 0) {
     // One item per CTA, clusters of csize consecutive CTAs (one unit each).
     cudaLaunchConfig_t cfg = {};
@@ -680,10 +690,12 @@ int launch_prefill(const Problem& pr, const Plan& pl, DeviceInfo& dev, int csize
                    cudaStream_t stream) {
   const int deg = cap_degree(pr);
   if (pl.dch == 1)
-    return deg == 5 ? launch_prefill_d<1, 5>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
+    return deg == 3 ? launch_prefill_d<1, 3>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
+         : deg == 5 ? launch_prefill_d<1, 5>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
          : deg == 7 ? launch_prefill_d<1, 7>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
                     : launch_prefill_d<1, 0>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream);
-  return deg == 5 ? launch_prefill_d<2, 5>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
+  return deg == 3 ? launch_prefill_d<2, 3>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
+       : deg == 5 ? launch_prefill_d<2, 5>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
        : deg == 7 ? launch_prefill_d<2, 7>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
                   : launch_prefill_d<2, 0>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream);
 }

@@ -96,7 +96,7 @@ struct PrefillParams {
                          // shared memory instead of the workspace; 0 = workspace merge
   int causal, window;
   float logit_scale, cap_in, cap_out;
-  // Softcap with a fixed exponent base (cap_fixed = 1): the capped logits,
+  // Softcap with a fixed exponent base (cap_fixed = 1, softcap code 3): the capped logits,
   // in log2 units, lie in [-cap_out, cap_out], so p = 2^(y - cap_base) with
   // cap_base = cap_out - B stays in [2^(B - 2 cap_out), 2^B].  The host picks
   // B = max(16, 2 cap_out - 120) and sets cap_fixed only when B <= 64, so p
@@ -267,10 +267,13 @@ __device__ __forceinline__ int key_tile(const PfItem& it, int t, int j) {
   return (t == 0 ? it.kt0[0] : it.kt0[1]) + j;
 }
 
-// kCapDeg: 0 = no softcap; 5 or 7 = softcap, with the odd polynomial of that
-// degree for tanh of small arguments (5 where the cap is small enough for its
-// error, see kTanh5C*).  kSplit: items cover key-range splits (splits > 1),
-// whose partials are merged; without it the split code is not compiled in.
+// kCapDeg: 0 = no softcap; 5 or 7 = softcap with the row max, with the odd
+// polynomial of that degree for tanh of small arguments (5 where the cap is
+// small enough for its error, see kTanh5C*); 3 = softcap with the degree-5
+// polynomial and a fixed exponent base (PrefillParams::cap_fixed), the only
+// softmax path compiled into that kernel.  kSplit: items cover key-range
+// splits (splits > 1), whose partials are merged; without it the split code
+// is not compiled in.
 template <int DCH, int kCapDeg, bool kSplit>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -650,8 +653,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         // the warp's rows is <= 1/2, tanh runs as an odd polynomial on the
         // FMA pipe).  On tiles with a mask the hidden scores become -inf and
         // are written back, so pass 2 is the same code on every tile.
-        if constexpr (kCapDeg == 5) {
-          if (p.cap_fixed) {
+        if constexpr (kCapDeg == 3) {
+          {
             // One pass over the scores, no row max: y = cap(x) - cap_base.
             // Per 32-key group, the warp takes the degree-5 polynomial when
             // every |x * cap_in| <= 1/2 (hidden keys as -inf then give p = 0),
@@ -907,8 +910,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       // meet at a named barrier below, so a warpgroup that gave up on a wait
       // still goes there (with ok = false) instead of leaving at once.
       // Fixed-base softcap: a row without a visible key keeps m = -inf.
-      if constexpr (kCapDeg == 5)
-        if (p.cap_fixed && !(l > 0.f)) m = -INFINITY;
+      if constexpr (kCapDeg == 3)
+        if (!(l > 0.f)) m = -INFINITY;
       const bool pair_x = kSplit && it.paired;
       if (!ok && !pair_x) break;
       // ---- epilogue.  The next item's first P.V of this tile may overwrite
