@@ -37,12 +37,12 @@ struct DeviceInfo {
   int sms = 0, major = 0, minor = 0;
   int smem_optin = 0;
   bool decode_attr[10] = {};  // per instantiation: [0, 8) 3/2-stage, [8, 10) 5-stage
-  bool prefill_attr[16] = {};  // per (DCH, softcap code, split) instantiation
+  bool prefill_attr[24] = {};  // per (DCH, softcap code, split mode) instantiation
   int append_blocks[4] = {};    // resident kv_append blocks per SM, per instantiation
   bool append_runs_ready[4] = {};  // staged-runs kernel's smem attribute set
   // Clusters of n CTAs of a split instantiation that can be resident at once
   // (cudaOccupancyMaxActiveClusters); -1 = not asked yet.
-  int cluster_max[16][9];
+  int cluster_max[24][9];
   DeviceInfo() {
     for (auto& a : cluster_max)
       for (int& n : a) n = -1;
@@ -523,15 +523,17 @@ int cap_degree(const Problem& pr) {
   return fixed ? 3 : 5;
 }
 
-template <int DCH, int kCapDeg, bool kSplit>
+// kSplit: 0 = no key splits, 1 = splits merged through the workspace,
+// 2 = paired splits merged inside a cluster.
+template <int DCH, int kCapDeg, int kSplit>
 constexpr int prefill_slot() {
   return (DCH - 1) + 2 * (kCapDeg == 5 ? 1 : kCapDeg == 7 ? 2 : kCapDeg == 3 ? 3 : 0) +
-         (kSplit ? 8 : 0);
+         8 * kSplit;
 }
 
 // One-time per device and instantiation (under g_mu): the register-split
 // check and the dynamic shared memory limit.
-template <int DCH, int kCapDeg, bool kSplit>
+template <int DCH, int kCapDeg, int kSplit>
 int prefill_setup(DeviceInfo& dev) {
   using C = PrefillCfg<DCH>;
   constexpr int attr = prefill_slot<DCH, kCapDeg, kSplit>();
@@ -566,9 +568,9 @@ int prefill_cluster_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, int* c
   if (!pl.split_pairs || g_no_cluster.load()) return GQA_ATTN_OK;
   const int half = pl.splits / 2;
   if (half < 2 || half > 8 || pl.ctas != pr.units * half) return GQA_ATTN_OK;
-  int rc = prefill_setup<DCH, kCapDeg, true>(dev);
+  int rc = prefill_setup<DCH, kCapDeg, 2>(dev);
   if (rc != GQA_ATTN_OK) return rc;
-  constexpr int attr = prefill_slot<DCH, kCapDeg, true>();
+  constexpr int attr = prefill_slot<DCH, kCapDeg, 2>();
   std::lock_guard<std::mutex> lk(g_mu);
   int& fit = dev.cluster_max[attr][half];
   if (fit < 0) {
@@ -584,7 +586,7 @@ int prefill_cluster_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, int* c
     cfg.attrs = at;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, prefill_sm100_kernel<DCH, kCapDeg, true>, &cfg) !=
+    if (cudaOccupancyMaxActiveClusters(&n, prefill_sm100_kernel<DCH, kCapDeg, 2>, &cfg) !=
         cudaSuccess) {
       (void)cudaGetLastError();
       n = 0;
@@ -608,7 +610,7 @@ int prefill_cluster(const Problem& pr, const Plan& pl, DeviceInfo& dev, int* csi
                   : prefill_cluster_k<2, 0>(pr, pl, dev, csize);
 }
 
-template <int DCH, int kCapDeg, bool kSplit>
+template <int DCH, int kCapDeg, int kSplit>
 int launch_prefill_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, int csize,
                      const void* q, const void* k, const void* v, void* o, void* ws,
                      void* tickets, cudaStream_t stream) {
@@ -640,7 +642,7 @@ int launch_prefill_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, int csi
   p.tickets = (unsigned int*)tickets;
   p.pair_heads = pl.pair_heads;
   p.heavy_first = (pr.causal || pr.window > 0) && !pl.split_pairs ? 1 : 0;
-  p.cluster_merge = kSplit ? csize : 0;
+  p.cluster_merge = kSplit == 2 ? csize : 0;
   p.causal = pr.causal;
   p.window = pr.window;
   const float rs = 1.0f / std::sqrt((float)pr.d);
@@ -650,7 +652,7 @@ int launch_prefill_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, int csi
   // Fixed exponent base (softcap code 3, see PrefillParams and cap_degree).
   p.cap_fixed = kCapDeg == 3 ? 1 : 0;
   p.cap_base = kCapDeg == 3 ? p.cap_out - cap_base_offset(p.cap_out) : 0.f;
-  if (p.cluster_merge > 0) {
+  if constexpr (kSplit == 2) {
     // One item per CTA, clusters of csize consecutive CTAs (one unit each).
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute at[1];
@@ -680,9 +682,11 @@ template <int DCH, int kCapDeg>
 int launch_prefill_d(const Problem& pr, const Plan& pl, DeviceInfo& dev, int csize,
                      const void* q, const void* k, const void* v, void* o, void* ws,
                      void* tickets, cudaStream_t stream) {
-  return pl.splits > 1
-             ? launch_prefill_k<DCH, kCapDeg, true>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream)
-             : launch_prefill_k<DCH, kCapDeg, false>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream);
+  if (pl.splits <= 1)
+    return launch_prefill_k<DCH, kCapDeg, 0>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream);
+  if (csize > 0)
+    return launch_prefill_k<DCH, kCapDeg, 2>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream);
+  return launch_prefill_k<DCH, kCapDeg, 1>(pr, pl, dev, csize, q, k, v, o, ws, tickets, stream);
 }
 
 int launch_prefill(const Problem& pr, const Plan& pl, DeviceInfo& dev, int csize, const void* q,

@@ -179,11 +179,11 @@ struct PfItem {
   bool busy;
 };
 
-template <bool kSplit>
+template <int kSplit>
 __device__ __forceinline__ PfItem prefill_item(const PrefillParams& p, const MaskSpec& ms,
                                                int item) {
   PfItem it;
-  it.paired = kSplit && p.split_pairs != 0;
+  it.paired = kSplit == 2 || (kSplit == 1 && p.split_pairs != 0);
   if (it.paired) {
     const int half = p.splits / 2;
     it.split = 2 * (item % half);
@@ -271,10 +271,12 @@ __device__ __forceinline__ int key_tile(const PfItem& it, int t, int j) {
 // polynomial of that degree for tanh of small arguments (5 where the cap is
 // small enough for its error, see kTanh5C*); 3 = softcap with the degree-5
 // polynomial and a fixed exponent base (PrefillParams::cap_fixed), the only
-// softmax path compiled into that kernel.  kSplit: items cover key-range
-// splits (splits > 1), whose partials are merged; without it the split code
-// is not compiled in.
-template <int DCH, int kCapDeg, bool kSplit>
+// softmax path compiled into that kernel.  kSplit: 0 = no key splits (the
+// split code is not compiled in); 1 = items cover key-range splits whose
+// partials are merged through the workspace; 2 = paired splits, one item
+// per CTA, merged inside a thread-block cluster.  Each kernel holds only its
+// own merge code: the workspace path alone made the clustered kernel slower.
+template <int DCH, int kCapDeg, int kSplit>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -1014,7 +1016,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           // Cluster merge: the partial stays in this CTA's shared memory (the
           // K/V ring and staging area are idle after the CTA's only item): O
           // as fp32 rows of d_pad + 4 floats, m and l per row.
-          const bool to_smem = paired && p.cluster_merge > 0;
+          const bool to_smem = kSplit == 2;
           if (quarter * 32 < wt.nrows && cw0 < cw1) {
             // Tile A = this warpgroup's (paired: t = 0) or the only tile.
             const int act_a = paired ? it.kc[0] : act, act_b = paired ? it.kc[1] : 0;
@@ -1183,7 +1185,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   // softmax warps of CTA `rank` merge column groups [g0, g1) of every row
   // from the partials of all CTAs of the cluster, in rank order.
   if constexpr (kSplit) {
-    if (p.cluster_merge > 0) {
+    if constexpr (kSplit == 2) {
       __syncwarp();
       cluster_sync();
       if (warp >= 4) {
