@@ -93,11 +93,12 @@ extern "C" {
  * and retires the old one without freeing it, so a CUDA graph captured
  * earlier on that stream keeps valid pointers; gqa_attn_release_workspace
  * frees everything.  Partials of the split-KV decode kernel and of the
- * tcgen05 kernel's key splits use the workspace; when every (batch, kv head)
- * has one 128-row tile split into 2 to 8 CTAs and all of the grid's CTAs fit
- * on the device at once, the tcgen05 kernel is launched as one thread-block
- * cluster per (batch, kv head), merges its partials in distributed shared
- * memory and allocates no workspace (gqa_attn_describe_merge tells which).
+ * tcgen05 kernel's key splits use the workspace.  The last CTA of a unit to
+ * finish merges them, except when every (batch, kv head) has one 128-row
+ * tile split into 2 to 8 CTAs and all of the grid's CTAs fit on the device
+ * at once: then the tcgen05 kernel is launched as one thread-block cluster
+ * per (batch, kv head), whose CTAs meet at the cluster barrier and merge a
+ * column slice each (gqa_attn_describe_merge tells which).
  *
  * CUDA graphs: a call of a given size on a stream enqueues only kernels (and
  * allocates nothing) once a call of that size has run on that stream, so
@@ -145,10 +146,10 @@ int gqa_attn_describe(int batch, int q_len, int kv_len, int num_q_heads, int num
  * key 2: force the number of key tiles per decode split (0 = automatic);
  * key 3: force the number of key splits of the tcgen05 kernel for units with
  *        one row tile (rounded up to even; 0 = automatic);
- * key 4: how those splits merge (0 = automatic: through distributed shared
- *        memory in one thread-block cluster per unit when a unit has 2 to 8
- *        CTAs and the whole grid fits on the device at once; -1 = always
- *        through the workspace);
+ * key 4: how those splits merge (0 = automatic: by every CTA of one
+ *        thread-block cluster per unit when a unit has 2 to 8 CTAs and the
+ *        whole grid fits on the device at once; -1 = always by the last CTA
+ *        of a unit to finish);
  * key 5: 1 = the tcgen05 kernel's softcap path always finds the row max
  *        before the exponentials (0 = automatic: caps up to about 63.8 use a
  *        fixed exponent base and a single pass over the scores).

@@ -141,8 +141,8 @@ def set_override(key: str, value: int) -> None:
     """Test/tuning knob: ``force_path`` (0 auto, 1 decode, 2 prefill),
     ``tiles_per_split`` (decode, 0 = automatic), ``prefill_splits``
     (tcgen05 kernel, units with one row tile; 0 = automatic) or
-    ``prefill_cluster`` (how those splits merge: 0 automatic, -1 always
-    through the workspace instead of a thread-block cluster) or
+    ``prefill_cluster`` (how those splits merge: 0 automatic, -1 always by
+    the last CTA of a unit instead of a thread-block cluster) or
     ``softcap_two_pass`` (1: the tcgen05 softcap path takes the row max
     first instead of its fixed exponent base)."""
     k = {"force_path": 1, "tiles_per_split": 2, "prefill_splits": 3, "prefill_cluster": 4,

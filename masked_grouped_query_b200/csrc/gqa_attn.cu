@@ -558,9 +558,10 @@ int prefill_setup(DeviceInfo& dev) {
 }
 
 // Paired key splits, one item per CTA: a cluster per unit merges its
-// partials through distributed shared memory when every cluster of the grid
-// can be resident at once (one wave) and a unit has 2..8 CTAs; *csize gets
-// the CTAs per cluster, or 0 for the workspace merge.
+// partials (every CTA a column slice, after the cluster barrier) when every
+// cluster of the grid can be resident at once (one wave) and a unit has 2..8
+// CTAs; *csize gets the CTAs per cluster, or 0 for the merge by the last CTA
+// of a unit (ticket).
 template <int DCH, int kCapDeg>
 int prefill_cluster_k(const Problem& pr, const Plan& pl, DeviceInfo& dev, int* csize) {
   using C = PrefillCfg<DCH>;
@@ -762,7 +763,8 @@ int run(const Problem& pr, const void* q, const void* k, const void* v, void* o,
                                                                  : GQA_ATTN_ERR_LAUNCH;
     }
     default: {
-      // Key splits merged in distributed shared memory need no workspace.
+      // Key splits merge through the workspace: by the last CTA of a unit to
+      // finish (ticket), or by all CTAs of the unit's cluster together.
       int csize = 0;
       if (pl.path == kPathPrefill && pl.splits > 1) {
         rc = prefill_cluster(pr, pl, *dev, &csize);
@@ -770,7 +772,7 @@ int run(const Problem& pr, const void* q, const void* k, const void* v, void* o,
       }
       void* ws = nullptr;
       void* tickets = nullptr;
-      if (pl.ws_bytes && csize == 0) {
+      if (pl.ws_bytes) {
         rc = get_workspace(stream, pl.ws_bytes, pl.ticket_bytes, &ws, &tickets);
         if (rc != GQA_ATTN_OK) return rc;
       }

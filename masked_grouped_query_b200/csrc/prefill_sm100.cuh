@@ -1013,10 +1013,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             return reinterpret_cast<float4*>(p.ws_o + (blk + sp) * (long long)p.d_pad * kPfM);
           };
           auto ml_of = [&](int sp) { return p.ws_ml + ((blk + sp) * 2 + hh) * 2 * kPfM; };
-          // Cluster merge: the partial stays in this CTA's shared memory (the
-          // K/V ring and staging area are idle after the CTA's only item): O
-          // as fp32 rows of d_pad + 4 floats, m and l per row.
-          const bool to_smem = kSplit == 2;
           if (quarter * 32 < wt.nrows && cw0 < cw1) {
             // Tile A = this warpgroup's (paired: t = 0) or the only tile.
             const int act_a = paired ? it.kc[0] : act, act_b = paired ? it.kc[1] : 0;
@@ -1031,7 +1027,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const float L = wa * la + (hb ? wb * lb : 0.f);
             const int ua = paired ? 0 : t;  // TMEM O of tile A
             float4* po = po_of(psplit);
-            float* crow = reinterpret_cast<float*>(ring) + r * (p.d_pad + 4);
             for (int c0 = cw0; c0 < cw1; c0 += 16) {
               float v[16];
 #pragma unroll
@@ -1051,19 +1046,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 #pragma unroll
               for (int g = 0; g < 4; ++g) {
                 const float4 f = make_float4(v[4 * g], v[4 * g + 1], v[4 * g + 2], v[4 * g + 3]);
-                if (to_smem)
-                  *reinterpret_cast<float4*>(crow + c0 + 4 * g) = f;
-                else
-                  po[(c0 / 4 + g) * kPfM + r] = f;
+                po[(c0 / 4 + g) * kPfM + r] = f;
               }
             }
-            float* pml = to_smem ? reinterpret_cast<float*>(stage_all) : ml_of(psplit);
-            if (!to_smem || t == 0) {
-              pml[r] = ha || hb ? mc : -INFINITY;
-              pml[kPfM + r] = L;
-            }
+            float* pml = ml_of(psplit);
+            pml[r] = ha || hb ? mc : -INFINITY;
+            pml[kPfM + r] = L;
           }
-          if (!to_smem) {
+          if constexpr (kSplit == 1) {
             // The ticket: every thread's partial is visible device-wide before
             // one thread of the warpgroup counts it (bounded waits: a warp that
             // gave up elsewhere makes the others give up here, not hang).
@@ -1180,10 +1170,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   }
 
   // ---------------------------------------------------------------- cluster merge
-  // Every thread of every CTA reaches both cluster barriers (no role leaves
-  // the kernel early; all waits above are bounded).  Between them the
+  // Every thread of every CTA reaches the cluster barrier (no role leaves the
+  // kernel early; all waits above are bounded).  Its release / acquire makes
+  // every CTA's partial in the workspace visible to the cluster; then the
   // softmax warps of CTA `rank` merge column groups [g0, g1) of every row
-  // from the partials of all CTAs of the cluster, in rank order.
+  // from the partials of all CTAs of the cluster, in rank order, reading
+  // them from L2.
   if constexpr (kSplit) {
     if constexpr (kSplit == 2) {
       __syncwarp();
@@ -1195,13 +1187,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const int g0 = (int)rank * G / csize, g1 = ((int)rank + 1) * G / csize, ng = g1 - g0;
         const int nrows = min(kPfM, p.rows);
         const int unit = (int)blockIdx.x / csize;
-        const int stride = p.d_pad + 4;
-        const float* cpart = reinterpret_cast<const float*>(ring);
-        const float* cml = reinterpret_cast<const float*>(stage_all);
+        const long long blk = (long long)unit * csize;  // the unit's partial slots
+        // Consecutive threads take consecutive rows: coalesced partial loads.
         for (int i = threadIdx.x - 128; i < nrows * ng; i += 256) {
-          const int row = i / ng, g = g0 + i % ng;
-          // Every peer's m, l and O values of this row and column group,
-          // all loads in flight together; then the weighted sum in rank order.
+          const int row = i % nrows, g = g0 + i / nrows;
           float mv[8], lv[8];
           float4 f[8];
 #pragma unroll
@@ -1210,9 +1199,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             lv[c] = 0.f;
             f[c] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (c < csize) {
-              mv[c] = ld_dsmem(dsmem_addr(cml + row, c));
-              lv[c] = ld_dsmem(dsmem_addr(cml + kPfM + row, c));
-              f[c] = ld_dsmem_v4(dsmem_addr(cpart + row * stride + 4 * g, c));
+              const float* ml = p.ws_ml + (blk + c) * 2 * 2 * kPfM;
+              mv[c] = __ldcg(ml + row);
+              lv[c] = __ldcg(ml + kPfM + row);
+              f[c] = __ldcg(reinterpret_cast<const float4*>(p.ws_o + (blk + c) * (long long)p.d_pad * kPfM) +
+                            g * kPfM + row);
             }
           }
           float M = -INFINITY;
@@ -1237,8 +1228,6 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           }
         }
       }
-      __syncwarp();
-      cluster_sync();  // the peers have read this CTA's partial
     }
   }
 

@@ -118,32 +118,12 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   return r;
 }
 
-// Every thread of every CTA in the cluster: shared-memory writes before it
-// are visible to the cluster's readers after it.  Not bounded: callers reach
+// Every thread of every CTA in the cluster: memory writes before it are
+// visible to the cluster's readers after it (release / acquire).  Not bounded: callers reach
 // it on every path (no thread leaves the kernel before it).
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
                    : "memory");
-}
-
-// Address of this CTA's shared variable `p` in the CTA of cluster rank `rank`.
-__device__ __forceinline__ uint32_t dsmem_addr(const void* p, uint32_t rank) {
-  uint32_t a;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
-  return a;
-}
-__device__ __forceinline__ float ld_dsmem(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ float4 ld_dsmem_v4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(addr)
-               : "memory");
-  return v;
 }
 
 // 3-D tiled bulk tensor store shared -> global, bulk-group completion.

@@ -262,9 +262,9 @@ def test_tcgen05_key_splits(cfg):
 ])
 def test_paired_split_merges(cfg):
     # Units with one row tile take two key splits per CTA; the partials
-    # merge through a cluster's distributed shared memory (automatic) or
-    # through the workspace (forced).  Both against the oracle, each
-    # deterministic, and the two within rounding of each other.
+    # merge by all CTAs of the unit's cluster after the cluster barrier
+    # (automatic) or by the last CTA to finish (forced).  Both against the
+    # oracle, each deterministic, and the two within rounding of each other.
     b, lq, lk, hq, hkv, d, causal, window, cap = cfg
     w = Workload("pm", b, lq, lk, hq, hkv, d, causal, window, cap, seed=lk + 3 * d)
     q, k, v = make_inputs(w)
