@@ -196,12 +196,21 @@ __device__ __forceinline__ PfItem prefill_item(const PrefillParams& p, const Mas
     ti.kr = key_range(ms, ti.row0, ti.nrows, kPfN);
     it.tile[0] = ti;
     it.tile[1] = ti;
-    const int per = (ti.kr.t_count + p.splits - 1) / p.splits;
+    // Split s takes key tiles [ceil(s T / S), ceil((s + 1) T / S)): sizes
+    // differ by at most one.  Tile A takes the larger of the item's two.
+    const int T = ti.kr.t_count, S = p.splits;
     for (int t = 0; t < 2; ++t) {
-      const int js = min(ti.kr.t_count, (it.split + t) * per);
-      const int je = min(ti.kr.t_count, js + per);
+      const int sp = it.split + t;
+      const int js = (sp * T + S - 1) / S, je = ((sp + 1) * T + S - 1) / S;
       it.kt0[t] = ti.kr.t_first + js;
       it.kc[t] = je - js;
+    }
+    if (it.kc[1] > it.kc[0]) {
+      const int k0 = it.kt0[0], c0 = it.kc[0];
+      it.kt0[0] = it.kt0[1];
+      it.kc[0] = it.kc[1];
+      it.kt0[1] = k0;
+      it.kc[1] = c0;
     }
     it.j_first = it.kt0[0];
     it.j_count = it.kc[0];  // kc[0] >= kc[1]
