@@ -253,8 +253,9 @@ __device__ __forceinline__ PfItem prefill_item(const PrefillParams& p, const Mas
     it.j_count = max(la, lb) - it.j_first + 1;
   }
   if (kSplit && p.splits > 1) {  // this item's share of the key tiles
-    const int per = (it.j_count + p.splits - 1) / p.splits;
-    const int js = min(it.j_count, it.split * per), je = min(it.j_count, js + per);
+    // Split s takes [ceil(s J / S), ceil((s + 1) J / S)) of the item's J.
+    const int J = it.j_count, S = p.splits;
+    const int js = (it.split * J + S - 1) / S, je = ((it.split + 1) * J + S - 1) / S;
     it.j_first += js;
     it.j_count = je - js;
   }
