@@ -259,6 +259,7 @@ def test_tcgen05_key_splits(cfg):
     (8, 4, 32768, 64, 4, 128, True, 4096, 30.0),   # 4 CTAs per unit
     (1, 3, 1000, 16, 1, 72, False, 300, None),     # 2 CTAs per unit, D = 72
     (3, 2, 777, 32, 2, 64, True, None, 20.0),      # 4 CTAs per unit, D = 64
+    (40, 4, 1000, 16, 1, 128, True, None, None),   # 3 CTAs per unit: uneven column slices
 ])
 def test_paired_split_merges(cfg):
     # Units with one row tile take two key splits per CTA; the partials
