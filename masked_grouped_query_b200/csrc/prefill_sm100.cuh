@@ -680,14 +680,11 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const f2 q2 = f2_pack(cc * ci2 * ci2 * kTanh5C5, cc * ci2 * ci2 * kTanh5C5);
             f2 acc[4] = {0ull, 0ull, 0ull, 0ull};
             auto group = [&](uint32_t(&sv)[32], int g) {
-              float mx = fmaxf(__uint_as_float(sv[0]), __uint_as_float(sv[1]));
-              float mn = fminf(__uint_as_float(sv[0]), __uint_as_float(sv[1]));
+              float am = fmaxf(fabsf(__uint_as_float(sv[0])), fabsf(__uint_as_float(sv[1])));
 #pragma unroll
-              for (int c = 2; c < 32; c += 2) {
-                mx = fmax3(mx, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
-                mn = fmin3(mn, __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
-              }
-              const bool poly = __all_sync(0xffffffffu, fmaxf(mx, -mn) * p.cap_in <= 0.5f);
+              for (int c = 2; c < 32; c += 2)
+                am = fmax3(am, fabsf(__uint_as_float(sv[c])), fabsf(__uint_as_float(sv[c + 1])));
+              const bool poly = __all_sync(0xffffffffu, am * p.cap_in <= 0.5f);
               if (need_mask) {
 #pragma unroll
                 for (int c = 0; c < 32; ++c)
@@ -765,14 +762,9 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             tmem_ld32(s_tm + 32 * g, sr);
             tmem_ld_wait();
             if constexpr (kCap) {
-              float mx = fmaxf(__uint_as_float(sr[0]), __uint_as_float(sr[1]));
-              float mn = fminf(__uint_as_float(sr[0]), __uint_as_float(sr[1]));
 #pragma unroll
-              for (int c = 2; c < 32; c += 2) {
-                mx = fmax3(mx, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-                mn = fmin3(mn, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
-              }
-              amax = fmax3(amax, mx, -mn);
+              for (int c = 0; c < 32; c += 2)
+                amax = fmax3(amax, fabsf(__uint_as_float(sr[c])), fabsf(__uint_as_float(sr[c + 1])));
             }
             if (need_mask) {
 #pragma unroll
