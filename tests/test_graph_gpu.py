@@ -17,8 +17,13 @@ pytestmark = pytest.mark.gpu
 @pytest.mark.parametrize("w", [
     Workload("decode", 4, 1, 3000, 32, 8, 128, True, None, None, 31),         # split-KV decode
     Workload("prefill", 1, 300, 900, 8, 2, 128, True, 256, 30.0, 32),         # tcgen05, key splits
+    Workload("clustered", 8, 4, 5000, 64, 4, 128, True, 2048, 30.0, 33),      # 4-CTA cluster merge
 ])
 def test_captured_call_replays_like_a_direct_call(w):
+    if w.name == "clustered":  # the cluster merge also writes its partials to the workspace
+        plan = mgq.describe(w.batch, w.q_len, w.kv_len, w.num_q_heads, w.num_kv_heads,
+                            w.head_dim, w.causal, w.window, w.softcap)
+        assert plan["cluster"] >= 2, plan
     q, k, v = (t.cuda() for t in make_inputs(w))
     out = torch.empty_like(q)
     s = torch.cuda.Stream()
