@@ -92,8 +92,9 @@ struct PrefillParams {
   int pair_heads;        // 1: tiles (2p, 2p+1) are two heads at one position
   int heavy_first;       // 1: items run in order of decreasing key-tile count (causal / window)
   int cluster_merge;     // paired items, one per CTA, launched as clusters of this many CTAs
-                         // (one cluster per unit): partials merge through distributed
-                         // shared memory instead of the workspace; 0 = workspace merge
+                         // (one cluster per unit): after one cluster barrier every CTA
+                         // merges a column slice of the unit's partials from the
+                         // workspace; 0 = the last CTA of a unit merges (tickets)
   int causal, window;
   float logit_scale, cap_in, cap_out;
   // Softcap with a fixed exponent base (cap_fixed = 1, softcap code 3): the capped logits,
@@ -283,9 +284,10 @@ __device__ __forceinline__ int key_tile(const PfItem& it, int t, int j) {
 // polynomial and a fixed exponent base (PrefillParams::cap_fixed), the only
 // softmax path compiled into that kernel.  kSplit: 0 = no key splits (the
 // split code is not compiled in); 1 = items cover key-range splits whose
-// partials are merged through the workspace; 2 = paired splits, one item
-// per CTA, merged inside a thread-block cluster.  Each kernel holds only its
-// own merge code: the workspace path alone made the clustered kernel slower.
+// partials the last CTA of a unit merges (tickets); 2 = paired splits, one
+// item per CTA, merged by the unit's thread-block cluster.  Both keep their
+// partials in the workspace.  Each kernel holds only its own merge code:
+// the ticket merge alone made the clustered kernel slower.
 template <int DCH, int kCapDeg, int kSplit>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
