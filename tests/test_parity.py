@@ -319,3 +319,28 @@ def test_clear_status_then_split_calls_match_oracle():
 def test_no_bounded_wait_expired():
     torch.cuda.synchronize()
     assert mgq.status() & 0x1f == 0
+
+
+@pytest.mark.parametrize("tiles,splits", [(8, 6), (11, 8)])
+@pytest.mark.parametrize("merge", [0, -1])
+def test_uneven_paired_splits(tiles, splits, merge):
+    # Split s of S takes key tiles [ceil(s T / S), ceil((s + 1) T / S)).  For
+    # these (T, S) some paired item's second split is the larger one (8 in 6:
+    # sizes 2 1 | 1 2 | 1 1), so its tile A takes that split instead.  Both
+    # merges (cluster, and last CTA with key 4 = -1) against the oracle.
+    w = Workload("us", 2, 4, tiles * 128, 16, 1, 128, False, None, None, seed=10 * tiles + splits)
+    q, k, v = make_inputs(w)
+    want = oracle.attention(q, k, v, causal=False, window=None, softcap=None)
+    q, k, v = q.cuda(), k.cuda(), v.cuda()
+    try:
+        mgq.set_override("prefill_splits", splits)
+        mgq.set_override("prefill_cluster", merge)
+        plan = mgq.describe(2, 4, tiles * 128, 16, 1, 128)
+        assert plan["path"] == "prefill" and plan["splits"] == splits and plan["tiles"] == tiles, plan
+        assert (plan["cluster"] >= 2) if merge == 0 else (plan["cluster"] == 0), plan
+        a = mgq.attention(q, k, v)
+        torch.cuda.synchronize()
+        assert_close(a, want, f"{tiles} tiles in {splits} splits, merge {merge}")
+    finally:
+        mgq.set_override("prefill_splits", 0)
+        mgq.set_override("prefill_cluster", 0)
