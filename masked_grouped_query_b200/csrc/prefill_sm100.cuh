@@ -10,8 +10,10 @@
 // head ("TPU v6e Masked GQA Kernel Optimization", "What You Have": GQA
 // ratios 1:1 to 16:1), so its K/V tiles are read once for all of them.
 //
-// Persistent: one CTA per SM walks the items blockIdx.x, blockIdx.x +
-// gridDim.x, ...; TMEM, barriers and the K/V ring live across items, and the
+// Persistent: one CTA per SM walks one item per round of gridDim.x items
+// (blockIdx.x of each round, or its mirror image on odd rounds when the items
+// are sorted heavy first: snake_item); TMEM, barriers and the K/V ring live
+// across items, and the
 // next item's Q is loaded as soon as the current item's last S = Q K^T has
 // been computed, so loads, MMAs and softmax of consecutive items overlap.
 //
@@ -266,6 +268,15 @@ __device__ __forceinline__ PfItem prefill_item(const PrefillParams& p, const Mas
   return it;
 }
 
+// The k-th item of this CTA in the persistent loop.  Items sorted heavy
+// first (causal / window) go out boustrophedon: round k hands item
+// k G + c to CTA c on even rounds and k G + (G - 1 - c) on odd ones, so no
+// CTA takes the heaviest item of every round.  The index grows with k.
+__device__ __forceinline__ int snake_item(const PrefillParams& p, int k) {
+  const int G = (int)gridDim.x, c = (int)blockIdx.x;
+  return k * G + ((p.heavy_first && (k & 1)) ? G - 1 - c : c);
+}
+
 __device__ __forceinline__ bool tile_active(const PfItem& it, int t, int j) {
   if (it.paired) return j < (t == 0 ? it.kc[0] : it.kc[1]);
   const KeyRange& kr = t == 0 ? it.tile[0].kr : it.tile[1].kr;
@@ -373,7 +384,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       int u = 0;       // K/V tiles issued (ring position, or stream position when paired)
       int nq = 0;      // busy items whose Q was issued
       bool ok = true;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      for (int kk = 0, item = snake_item(p, 0); item < p.n_items && ok;
+           ++kk, item = snake_item(p, kk)) {
         const PfItem it = prefill_item<kSplit>(p, ms, item);
         if (!it.busy) continue;
         const int kvh = it.unit % p.kv_heads, bidx = it.unit / p.kv_heads;
@@ -457,7 +469,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       int nq = 0;                 // busy items started (q_full phases)
       int n_act[2] = {0, 0};      // P tiles consumed per q tile (p_full phases)
       bool ok = true;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      for (int kk = 0, item = snake_item(p, 0); item < p.n_items && ok;
+           ++kk, item = snake_item(p, kk)) {
         const PfItem it = prefill_item<kSplit>(p, ms, item);
         if (!it.busy) continue;
         if (!(ok = mbar_wait(q_full, nq & 1, kStatusTimeoutMma))) break;
@@ -636,7 +649,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     int n_busy = 0;   // busy items finished (o_done phases)
     int n_merge = 0;  // split tickets taken by this warpgroup (part_done[t] phases)
     bool ok = true;
-    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+    for (int kk = 0, item = snake_item(p, 0); item < p.n_items && ok;
+         ++kk, item = snake_item(p, kk)) {
       const PfItem it = prefill_item<kSplit>(p, ms, item);
       const TileInfo ti = t ? it.tile[1] : it.tile[0];
       int lo = 0, hi = -1;  // visible keys of this row (hi < lo: none)
